@@ -1,0 +1,177 @@
+"""Python binding of libsdpa, the fused SDPA forward for B200 (sm_100a).
+
+Argument marshalling only: every step of the attention runs in the CUDA
+kernels of ``libsdpa.so`` behind the C ABI declared in ``include/sdpa.h``.
+PyTorch supplies device memory and the current stream.  There is no CPU
+fallback: importing works without a GPU (so the ABI can be inspected), but
+every call needs CUDA tensors and the built library, and raises otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsdpa.so")
+
+SDPA_F32, SDPA_BF16 = 0, 1
+MASK_NONE, MASK_CAUSAL, MASK_SLIDING, MASK_FLOAT, MASK_BOOL = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_EXACT, PATH_TCGEN05, PATH_SMALL_D, PATH_SPLIT_KV = 0, 1, 2, 3, 4
+PATHS = {"auto": PATH_AUTO, "exact": PATH_EXACT, "tcgen05": PATH_TCGEN05,
+         "small_d": PATH_SMALL_D, "split_kv": PATH_SPLIT_KV}
+STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
+          -3: "SDPA_ERR_MISALIGNED", -4: "SDPA_ERR_CUDA", -5: "SDPA_ERR_TIMEOUT",
+          -6: "SDPA_ERR_CAPACITY"}
+
+# Every symbol include/sdpa.h declares.
+EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_select_path", "sdpa_fwd_host",
+           "sdpa_last_device_error", "sdpa_strerror", "sdpa_version")
+
+
+class SdpaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}" if what else STATUS.get(status, str(status)))
+
+
+class sdpa_mask_t(ctypes.Structure):
+    _fields_ = [("offset", ctypes.c_int64), ("window", ctypes.c_int64), ("data", ctypes.c_void_p),
+                ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64), ("stride_q", ctypes.c_int64)]
+
+
+_lib = None
+_vp, _i32, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_COMMON = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32]
+
+
+def lib():
+    """The loaded ``libsdpa.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libsdpa.so is not built ({LIB_PATH}); run "
+                              "`python -m attention_sdpa_fwd_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.sdpa_fwd.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.sdpa_fwd_ex.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+        L.sdpa_fwd_host.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+        L.sdpa_select_path.argtypes = _COMMON + [_i32, _vp, _vp, _vp, _vp, _vp]
+        L.sdpa_last_device_error.argtypes = [_vp]
+        L.sdpa_strerror.argtypes = [_i32]
+        L.sdpa_strerror.restype = ctypes.c_char_p
+        for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_host", "sdpa_select_path",
+                     "sdpa_last_device_error", "sdpa_version"):
+            getattr(L, name).restype = _i32
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# Raw C-ABI calls (same names as the C functions; pointers are ints)
+# ---------------------------------------------------------------------------
+def _hw(x):
+    return None if x is None else (ctypes.c_int * 2)(int(x[0]), int(x[1]))
+
+
+def sdpa_fwd(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+             rel_pos_h, rel_pos_w, q_hw, k_hw, stream) -> int:
+    return lib().sdpa_fwd(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                          rel_pos_h, rel_pos_w, _hw(q_hw), _hw(k_hw), stream)
+
+
+def sdpa_fwd_ex(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                rel_pos_h, rel_pos_w, q_hw, k_hw, lse, path, stream) -> int:
+    return lib().sdpa_fwd_ex(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                             rel_pos_h, rel_pos_w, _hw(q_hw), _hw(k_hw), lse, path, stream)
+
+
+def sdpa_fwd_host(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                  rel_pos_h, rel_pos_w, q_hw, k_hw, path, stream) -> int:
+    return lib().sdpa_fwd_host(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                               rel_pos_h, rel_pos_w, _hw(q_hw), _hw(k_hw), path, stream)
+
+
+def sdpa_select_path(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, mask_kind, mask_ptr,
+                     rel_pos_h, rel_pos_w, q_hw, k_hw) -> int:
+    return lib().sdpa_select_path(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, mask_kind, mask_ptr,
+                                  rel_pos_h, rel_pos_w, _hw(q_hw), _hw(k_hw))
+
+
+def sdpa_last_device_error(stream) -> int:
+    return lib().sdpa_last_device_error(stream)
+
+
+def sdpa_strerror(status: int) -> str:
+    return lib().sdpa_strerror(status).decode()
+
+
+def sdpa_version() -> int:
+    return lib().sdpa_version()
+
+
+# ---------------------------------------------------------------------------
+# Tensor-level convenience wrapper (marshalling only)
+# ---------------------------------------------------------------------------
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return SDPA_F32
+    if t.dtype == torch.bfloat16:
+        return SDPA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def make_mask(kind: int, *, offset: int = 0, window: int = 0, tensor=None) -> Optional[sdpa_mask_t]:
+    """Build the host mask descriptor.  ``tensor`` (ADD_FLOAT / BOOL) must be a
+    CUDA tensor of 4 dims [B|1, Hq|1, Tq, Tkv] with a contiguous key axis;
+    size-1 batch / head axes broadcast (stride 0)."""
+    if kind == MASK_NONE:
+        return None
+    m = sdpa_mask_t(offset=int(offset), window=int(window), data=None, stride_b=0, stride_h=0, stride_q=0)
+    if kind in (MASK_FLOAT, MASK_BOOL):
+        t = tensor
+        if t is None or t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError("mask tensor must be 4-D with a contiguous last axis")
+        m.data = t.data_ptr()
+        m.stride_b = 0 if t.shape[0] == 1 else t.stride(0)
+        m.stride_h = 0 if t.shape[1] == 1 else t.stride(1)
+        m.stride_q = t.stride(2)
+    return m
+
+
+def sdpa(q, k, v, scale: Optional[float] = None, *, mask_kind: int = MASK_NONE, offset: int = 0,
+         window: int = 0, mask=None, rel_pos_h=None, rel_pos_w=None,
+         q_hw: Optional[Sequence[int]] = None, k_hw: Optional[Sequence[int]] = None,
+         out=None, lse=None, path: str = "auto", stream=None):
+    """softmax(q.k^T*scale + bias).v on CUDA tensors in bhsd layout.
+
+    q [B,Hq,Tq,d], k/v [B,Hkv,Tkv,d], contiguous, float32 or bfloat16.
+    ``scale`` defaults to 1/sqrt(d) (Axon PR, :scale option).  Returns ``out``."""
+    import torch
+    for t in (q, k, v):
+        if not t.is_cuda:
+            raise ValueError("sdpa runs on CUDA tensors only (no CPU fallback)")
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous (bhsd)")
+    B, Hq, Tq, d = q.shape
+    Hkv, Tkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    m = make_mask(mask_kind, offset=offset, window=window, tensor=mask)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = sdpa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, Hq, Hkv, Tq, Tkv, d,
+                         float(scale), mask_kind, ctypes.byref(m) if m is not None else None,
+                         _ptr(rel_pos_h), _ptr(rel_pos_w), q_hw, k_hw, _ptr(lse), PATHS[path],
+                         st.cuda_stream)
+    if rc != 0:
+        raise SdpaError(rc, "sdpa_fwd_ex")
+    return out

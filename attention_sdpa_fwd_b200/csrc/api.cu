@@ -1,0 +1,296 @@
+// C ABI of libsdpa: argument validation, kernel-family selection, launch.
+// Declarations and the meaning of every argument: include/sdpa.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace sdpa {
+
+// Bit set by kernels whose bounded waits expire; read and cleared by
+// sdpa_last_device_error().
+__device__ int g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int* error_word_ptr() {
+  static int* ptrs[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+struct Problem {
+  Params p;
+  sdpa_dtype_t dtype;
+  size_t esz;
+  bool empty_out;  // nothing to write
+};
+
+// Validates everything that can be checked on the host and fills the kernel
+// parameters.  Pointers are only checked for NULL, alignment to the element
+// size and overlap of `out` with the inputs.
+int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype, int B,
+                  int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
+                  const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
+                  const int* q_hw, const int* k_hw, float* lse, Problem* pr) {
+  memset(pr, 0, sizeof(*pr));
+  if (dtype != SDPA_F32 && dtype != SDPA_BF16) return SDPA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || Tq < 0 || Tkv < 0) return SDPA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SDPA_ERR_INVALID_ARG;
+  if (!(d == 16 || d == 64 || d == 128)) return SDPA_ERR_UNSUPPORTED;
+  if (!isfinite(scale)) return SDPA_ERR_INVALID_ARG;
+  if (mask_kind < SDPA_MASK_NONE || mask_kind > SDPA_MASK_BOOL) return SDPA_ERR_INVALID_ARG;
+  const size_t esz = dtype == SDPA_F32 ? 4 : 2;
+  Params& p = pr->p;
+  p.q = q; p.k = k; p.v = v; p.out = out; p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Tq = Tq; p.Tkv = Tkv; p.d = d;
+  p.group = Hq / Hkv;
+  p.scale = scale;
+  p.mask_kind = mask_kind;
+  const long long rows = (long long)B * Hq * Tq;
+  pr->empty_out = rows == 0;
+  pr->dtype = dtype;
+  pr->esz = esz;
+
+  const sdpa_mask_t* m = static_cast<const sdpa_mask_t*>(mask_ptr);
+  if (mask_kind == SDPA_MASK_CAUSAL) {
+    p.offset = m ? m->offset : 0;
+  } else if (mask_kind == SDPA_MASK_SLIDING) {
+    if (m == nullptr || m->window < 1) return SDPA_ERR_INVALID_ARG;
+    p.offset = m->offset;
+    p.window = m->window;
+  } else if (mask_kind == SDPA_MASK_ADD_FLOAT || mask_kind == SDPA_MASK_BOOL) {
+    if (m == nullptr) return SDPA_ERR_INVALID_ARG;
+    if (m->stride_b < 0 || m->stride_h < 0 || m->stride_q < 0) return SDPA_ERR_INVALID_ARG;
+    if (!pr->empty_out && Tkv > 0 && m->data == nullptr) return SDPA_ERR_INVALID_ARG;
+    const size_t mesz = mask_kind == SDPA_MASK_BOOL ? 1 : esz;
+    if (m->data && !aligned(m->data, mesz)) return SDPA_ERR_MISALIGNED;
+    p.mask = m->data;
+    p.msb = m->stride_b; p.msh = m->stride_h; p.msq = m->stride_q;
+  }
+  if (p.offset > (1LL << 40) || p.offset < -(1LL << 40) || p.window > (1LL << 40))
+    return SDPA_ERR_INVALID_ARG;
+
+  if ((rel_pos_h == nullptr) != (rel_pos_w == nullptr)) return SDPA_ERR_INVALID_ARG;
+  if (rel_pos_h != nullptr) {
+    if (q_hw == nullptr || k_hw == nullptr) return SDPA_ERR_INVALID_ARG;
+    if (q_hw[0] < 1 || q_hw[1] < 1 || k_hw[0] < 1 || k_hw[1] < 1) return SDPA_ERR_INVALID_ARG;
+    if ((long long)q_hw[0] * q_hw[1] != Tq || (long long)k_hw[0] * k_hw[1] != Tkv)
+      return SDPA_ERR_INVALID_ARG;
+    if (q_hw[0] != k_hw[0] || q_hw[1] != k_hw[1]) return SDPA_ERR_UNSUPPORTED;
+    if (!aligned(rel_pos_h, esz) || !aligned(rel_pos_w, esz)) return SDPA_ERR_MISALIGNED;
+    p.use_rel = 1;
+    p.rel_h = rel_pos_h; p.rel_w = rel_pos_w;
+    p.qh_n = q_hw[0]; p.qw_n = q_hw[1]; p.kh_n = k_hw[0]; p.kw_n = k_hw[1];
+  }
+
+  if (!pr->empty_out) {
+    if (q == nullptr || out == nullptr) return SDPA_ERR_INVALID_ARG;
+    if (Tkv > 0 && (k == nullptr || v == nullptr)) return SDPA_ERR_INVALID_ARG;
+    if (!aligned(q, esz) || !aligned(out, esz) || (k && !aligned(k, esz)) || (v && !aligned(v, esz)))
+      return SDPA_ERR_MISALIGNED;
+    if (lse && !aligned(lse, 4)) return SDPA_ERR_MISALIGNED;
+    const size_t nq = (size_t)rows * d * esz;
+    const size_t nk = (size_t)B * Hkv * Tkv * d * esz;
+    if (overlaps(out, nq, q, nq) || overlaps(out, nq, k, nk) || overlaps(out, nq, v, nk))
+      return SDPA_ERR_INVALID_ARG;
+    if (lse && (overlaps(lse, (size_t)rows * 4, out, nq) || overlaps(lse, (size_t)rows * 4, q, nq)))
+      return SDPA_ERR_INVALID_ARG;
+  }
+  p.k_vec16 = (k != nullptr && aligned(k, 16)) ? 1 : 0;
+  return SDPA_OK;
+}
+
+int choose_path(const Problem& pr) {
+  (void)pr;
+  return SDPA_PATH_EXACT;
+}
+
+int run(const Problem& pr, int path, cudaStream_t stream) {
+  if (pr.empty_out) return SDPA_OK;
+  Params p = pr.p;
+  p.err = error_word_ptr();
+  if (p.err == nullptr) return SDPA_ERR_CUDA;
+  if (path == SDPA_PATH_AUTO) path = choose_path(pr);
+  cudaError_t e;
+  switch (path) {
+    case SDPA_PATH_EXACT: e = launch_exact(p, pr.dtype, stream); break;
+    case SDPA_PATH_TCGEN05:
+    case SDPA_PATH_SMALL_D:
+    case SDPA_PATH_SPLIT_KV: return SDPA_ERR_UNSUPPORTED;
+    default: return SDPA_ERR_INVALID_ARG;
+  }
+  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sdpa
+
+using namespace sdpa;
+
+extern "C" int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                           int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
+                           const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
+                           const int* q_hw, const int* k_hw, float* lse, int path, cudaStream_t stream) {
+  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_SPLIT_KV) return SDPA_ERR_INVALID_ARG;
+  Problem pr;
+  int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                         rel_pos_h, rel_pos_w, q_hw, k_hw, lse, &pr);
+  if (rc != SDPA_OK) return rc;
+  return run(pr, path, stream);
+}
+
+extern "C" int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                        int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
+                        const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
+                        const int* q_hw, const int* k_hw, cudaStream_t stream) {
+  return sdpa_fwd_ex(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                     rel_pos_h, rel_pos_w, q_hw, k_hw, nullptr, SDPA_PATH_AUTO, stream);
+}
+
+extern "C" int sdpa_select_path(const void* q, const void* k, const void* v, void* out,
+                                sdpa_dtype_t dtype, int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                                int mask_kind, const void* mask_ptr, const void* rel_pos_h,
+                                const void* rel_pos_w, const int* q_hw, const int* k_hw) {
+  Problem pr;
+  int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, 1.0f, mask_kind, mask_ptr,
+                         rel_pos_h, rel_pos_w, q_hw, k_hw, nullptr, &pr);
+  if (rc != SDPA_OK) return rc;
+  return choose_path(pr);
+}
+
+
+namespace sdpa {
+namespace {
+
+// Device staging buffer of sdpa_fwd_host, one per device, grown on demand.
+struct Staging {
+  void* buf = nullptr;
+  size_t cap = 0;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+}  // namespace sdpa
+
+extern "C" int sdpa_fwd_host(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                             int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
+                             const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
+                             const int* q_hw, const int* k_hw, int path, cudaStream_t stream) {
+  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_SPLIT_KV) return SDPA_ERR_INVALID_ARG;
+  Problem pr;
+  int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                         rel_pos_h, rel_pos_w, q_hw, k_hw, nullptr, &pr);
+  if (rc != SDPA_OK) return rc;
+  if (pr.empty_out) return SDPA_OK;
+  static Staging staging[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SDPA_ERR_CUDA;
+
+  const size_t esz = pr.esz;
+  const size_t nq = (size_t)B * Hq * Tq * d * esz;
+  const size_t nk = (size_t)B * Hkv * Tkv * d * esz;
+  size_t nrh = 0, nrw = 0, nmask = 0;
+  if (pr.p.use_rel) {
+    nrh = (size_t)(2 * pr.p.kh_n - 1) * d * esz;
+    nrw = (size_t)(2 * pr.p.kw_n - 1) * d * esz;
+  }
+  const bool tensor_mask = mask_kind == SDPA_MASK_ADD_FLOAT || mask_kind == SDPA_MASK_BOOL;
+  if (tensor_mask && Tkv > 0) {
+    const size_t mesz = mask_kind == SDPA_MASK_BOOL ? 1 : esz;
+    const long long last = (long long)(B - 1) * pr.p.msb + (long long)(Hq - 1) * pr.p.msh +
+                           (long long)(Tq - 1) * pr.p.msq + Tkv;
+    nmask = (size_t)last * mesz;
+  }
+  const size_t oq = 0, ok = round_up(oq + nq, 256), ov = round_up(ok + nk, 256),
+               oo = round_up(ov + nk, 256), orh = round_up(oo + nq, 256),
+               orw = round_up(orh + nrh, 256), om = round_up(orw + nrw, 256),
+               total = round_up(om + nmask, 256);
+
+  std::lock_guard<std::mutex> lock(mu);
+  Staging& st = staging[dev];
+  if (st.cap < total) {
+    if (st.buf) cudaFree(st.buf);
+    st.buf = nullptr;
+    st.cap = 0;
+    if (cudaMalloc(&st.buf, total) != cudaSuccess) return SDPA_ERR_CUDA;
+    st.cap = total;
+  }
+  char* base = static_cast<char*>(st.buf);
+  auto h2d = [&](size_t off, const void* src, size_t n) {
+    return n == 0 || cudaMemcpyAsync(base + off, src, n, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+  };
+  if (!h2d(oq, q, nq) || !h2d(ok, k, nk) || !h2d(ov, v, nk) || !h2d(orh, rel_pos_h, nrh) ||
+      !h2d(orw, rel_pos_w, nrw))
+    return SDPA_ERR_CUDA;
+  sdpa_mask_t dmask;
+  const void* mptr = mask_ptr;
+  if (tensor_mask) {
+    dmask = *static_cast<const sdpa_mask_t*>(mask_ptr);
+    if (!h2d(om, dmask.data, nmask)) return SDPA_ERR_CUDA;
+    dmask.data = nmask ? base + om : nullptr;
+    mptr = &dmask;
+  }
+  Problem dpr;
+  rc = build_problem(base + oq, Tkv ? base + ok : nullptr, Tkv ? base + ov : nullptr, base + oo, dtype, B,
+                     Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mptr, nrh ? base + orh : nullptr,
+                     nrw ? base + orw : nullptr, q_hw, k_hw, nullptr, &dpr);
+  if (rc != SDPA_OK) return rc;
+  rc = run(dpr, path, stream);
+  if (rc != SDPA_OK) return rc;
+  if (cudaMemcpyAsync(out, base + oo, nq, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return SDPA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SDPA_ERR_CUDA;
+  return SDPA_OK;
+}
+
+extern "C" int sdpa_last_device_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SDPA_ERR_CUDA;
+  int* w = error_word_ptr();
+  if (w == nullptr) return SDPA_ERR_CUDA;
+  int host = 0;
+  if (cudaMemcpy(&host, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SDPA_ERR_CUDA;
+  if (host != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SDPA_ERR_CUDA;
+    return SDPA_ERR_TIMEOUT;
+  }
+  return SDPA_OK;
+}
+
+extern "C" const char* sdpa_strerror(int status) {
+  switch (status) {
+    case SDPA_OK: return "ok";
+    case SDPA_ERR_INVALID_ARG: return "invalid argument";
+    case SDPA_ERR_UNSUPPORTED: return "unsupported by this build";
+    case SDPA_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case SDPA_ERR_CUDA: return "CUDA error";
+    case SDPA_ERR_TIMEOUT: return "device-side wait timed out";
+    case SDPA_ERR_CAPACITY: return "request exceeds a fixed-size buffer";
+  }
+  return "unknown status";
+}
+
+extern "C" int sdpa_version(void) { return 100; }

@@ -1,0 +1,64 @@
+// Shared host/device definitions of libsdpa's kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sdpa.h"
+
+namespace sdpa {
+
+// Everything a kernel needs, filled on the host after validation.
+struct Params {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;        // optional [B, Hq, Tq]
+  int B, Hq, Hkv, Tq, Tkv, d;
+  int group;         // Hq / Hkv
+  float scale;
+  int mask_kind;
+  long long offset, window;
+  const void* mask;  // ADD_FLOAT (I/O dtype) or BOOL (uint8)
+  long long msb, msh, msq;
+  const void* rel_h;
+  const void* rel_w;
+  int use_rel;
+  int qh_n, qw_n, kh_n, kw_n;  // query / key patch grids (height, width)
+  int* err;          // device error word (bounded waits report here)
+  int k_vec16;       // k's base is 16-byte aligned (vector loads allowed)
+};
+
+enum ErrBits { ERR_WAIT_TIMEOUT = 1 };
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Visible key range [lo, hi) of query row i under CAUSAL / SLIDING; the whole
+// key axis otherwise.
+__host__ __device__ __forceinline__ void key_range(const Params& p, long long i, long long& lo,
+                                                   long long& hi) {
+  lo = 0;
+  hi = p.Tkv;
+  if (p.mask_kind == SDPA_MASK_CAUSAL || p.mask_kind == SDPA_MASK_SLIDING) {
+    long long top = i + p.offset + 1;  // exclusive upper bound
+    if (top < hi) hi = top;
+    if (p.mask_kind == SDPA_MASK_SLIDING) {
+      long long bot = i + p.offset - p.window + 1;
+      if (bot > lo) lo = bot;
+    }
+    if (hi < lo) hi = lo;
+  }
+}
+
+// Launchers (one per kernel family); each returns a cudaError_t of the launch.
+cudaError_t launch_exact(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
+
+}  // namespace sdpa

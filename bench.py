@@ -1,0 +1,428 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused SDPA forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--per-config]
+
+One step = one pass of the whole hot path over one batch: the fused forward
+(Q/K/V tiles in, rel-pos projections, QK^T, bias/mask, online softmax, PV,
+epilogue) on the SAM ViT-B global-attention workload (B=1, 12 heads, 64x64
+patch grid -> 4096 tokens, head_dim 64, bf16, decomposed rel-pos bias), with
+inputs resident in HBM.  Several independent input sets (together larger than
+the 126 MB L2) are cycled so consecutive steps never hit a warm L2.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own
+independent problem (weak scaling, no collective on the data path); the time
+is the max over ranks.
+
+Rank 0 prints ONE JSON line.  ``--impl reference`` times the fp64 CPU oracle
+(the slow, plain definition) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_sdpa_fwd_b200 import workloads as W  # noqa: E402
+
+METRIC = "attention TFLOP/s and % of B200 bf16 peak (or HBM GB/s %) per config, 1 GPU"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler (nvidia-smi during the timed region)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.samples:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        used = inside if inside else sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
+        if not used:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        mhz = sorted(r[1] for r in used)
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in used:
+            for n, v in zip(names, r[3][5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(r[2] for r in used),
+                "reasons": sorted(reasons), "samples": len(used), "samples_in_window": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "attention_sdpa_fwd_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_hash: str, workload: str):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, or None when absent or taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source_hash") != kernel_hash:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def make_device_sets(spec: W.Spec, device, nsets: int, seed_base: int):
+    sets = []
+    for s in range(nsets):
+        wl = W.make(spec, seed=seed_base + s)
+        t = lambda x: None if x is None else x.to(device, non_blocking=False).contiguous()
+        sets.append(dict(q=t(wl.q), k=t(wl.k), v=t(wl.v), rh=t(wl.rel_pos_h), rw=t(wl.rel_pos_w),
+                         mask=t(wl.mask), out=torch.empty_like(wl.q, device=device)))
+    return sets
+
+
+def launch(S, spec: W.Spec, st, stream, path):
+    m = S.make_mask(spec.mask_kind, offset=spec.offset, window=spec.window, tensor=st["mask"])
+    import ctypes
+    rc = S.sdpa_fwd_ex(st["q"].data_ptr(), st["k"].data_ptr(), st["v"].data_ptr(), st["out"].data_ptr(),
+                       S.SDPA_BF16 if spec.dtype == torch.bfloat16 else S.SDPA_F32,
+                       spec.B, spec.Hq, spec.Hkv, spec.Tq, spec.Tkv, spec.d, spec.scale, spec.mask_kind,
+                       ctypes.byref(m) if m is not None else None,
+                       st["rh"].data_ptr() if st["rh"] is not None else None,
+                       st["rw"].data_ptr() if st["rw"] is not None else None,
+                       spec.q_hw, spec.k_hw, None, path, stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"sdpa_fwd_ex failed: {S.STATUS.get(rc, rc)}")
+
+
+def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, ws: int, path=0):
+    per_set = spec.bytes()
+    nsets = max(2, math.ceil(2 * L2_BYTES / max(per_set, 1)))
+    nsets = min(nsets, 64)
+    sets = make_device_sets(spec, device, nsets, seed_base=spec.seed + 1000 * rank)
+    stream = torch.cuda.current_stream(device)
+    for i in range(warmup):
+        launch(S, spec, sets[i % nsets], stream, path)
+    torch.cuda.synchronize(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t0 = time.time()
+    e0.record(stream)
+    for i in range(steps):
+        starts[i].record(stream)
+        launch(S, spec, sets[i % nsets], stream, path)
+        ends[i].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    t1 = time.time()
+    if ws > 1:
+        torch.distributed.barrier()
+    total_ms = e0.elapsed_time(e1)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return dict(total_ms=total_ms, launch_ms=launch_ms, t0=t0, t1=t1, nsets=nsets,
+                set_bytes=per_set)
+
+
+def time_e2e(S, spec: W.Spec, device, steps: int, warmup: int):
+    """Same forward through the host-buffer C entry point: pinned host inputs,
+    H2D copies, kernel, D2H copy of the output, all inside the timed region."""
+    wl = W.make(spec, seed=spec.seed + 777)
+    pin = lambda x: None if x is None else x.contiguous().pin_memory()
+    q, k, v, rh, rw = (pin(x) for x in (wl.q, wl.k, wl.v, wl.rel_pos_h, wl.rel_pos_w))
+    out = torch.empty_like(q).pin_memory()
+    stream = torch.cuda.current_stream(device)
+    import ctypes
+    mask_h = pin(wl.mask)
+    m = None
+    if spec.mask_kind != W.MASK_NONE:
+        m = S.sdpa_mask_t(offset=spec.offset, window=spec.window, data=None, stride_b=0, stride_h=0, stride_q=0)
+        if mask_h is not None:
+            m.data = mask_h.data_ptr()
+            m.stride_b = 0 if mask_h.shape[0] == 1 else mask_h.stride(0)
+            m.stride_h = 0 if mask_h.shape[1] == 1 else mask_h.stride(1)
+            m.stride_q = mask_h.stride(2)
+
+    def call():
+        rc = S.sdpa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             S.SDPA_BF16 if spec.dtype == torch.bfloat16 else S.SDPA_F32,
+                             spec.B, spec.Hq, spec.Hkv, spec.Tq, spec.Tkv, spec.d, spec.scale, spec.mask_kind,
+                             ctypes.byref(m) if m is not None else None,
+                             rh.data_ptr() if rh is not None else None,
+                             rw.data_ptr() if rw is not None else None,
+                             spec.q_hw, spec.k_hw, 0, stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"sdpa_fwd_host failed: {S.STATUS.get(rc, rc)}")
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sum(x.numel() * x.element_size() for x in (q, k, v, rh, rw, mask_h) if x is not None)
+    d2h = out.numel() * out.element_size()
+    return ms, h2d, d2h
+
+
+def cpu_oracle_sample(spec: W.Spec, budget_s: float = 12.0):
+    """Time the fp64 oracle on the host cores on a bounded row sample."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    wl = W.make(spec)
+    kw = dict(mask_kind=spec.mask_kind, offset=spec.offset, window=spec.window)
+    if spec.mask_kind in (W.MASK_FLOAT, W.MASK_BOOL):
+        kw["mask"] = wl.mask
+    if spec.rel:
+        kw.update(rel_pos_h=wl.rel_pos_h, rel_pos_w=wl.rel_pos_w, q_hw=spec.q_hw, k_hw=spec.k_hw)
+    # probe with a small sample, then size the real one to about budget_s
+    probe = list(range(0, spec.Tq, max(1, spec.Tq // 16)))
+    t = time.time()
+    oracle.sdpa(wl.q, wl.k, wl.v, spec.scale, rows=probe, **kw)
+    dt = max(time.time() - t, 1e-4)
+    per_row = dt / len(probe)
+    nrows = int(min(spec.Tq, max(len(probe), budget_s / per_row)))
+    stride = max(1, spec.Tq // nrows)
+    rows = list(range(0, spec.Tq, stride))[:nrows]
+    t = time.time()
+    oracle.sdpa(wl.q, wl.k, wl.v, spec.scale, rows=rows, **kw)
+    sec = time.time() - t
+    frac = len(rows) / spec.Tq
+    flops = spec.flops() * frac
+    return dict(value=flops / sec / 1e12, unit="TFLOP/s", cores=oracle.num_threads(), kind="oracle",
+                sample=f"{spec.name}: all {spec.B * spec.Hq} (b,h) x {len(rows)} of {spec.Tq} query rows "
+                       f"(fp64, {sec:.1f} s)", seconds=sec)
+
+
+def run_ours(args):
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import attention_sdpa_fwd_b200 as S
+    from attention_sdpa_fwd_b200 import build
+    if rank == 0 or ws == 1:
+        pass
+    S.lib()  # fails loudly if the extension is missing
+    peaks, peaks_src = load_peaks()
+    spec = W.SPECS[args.workload]
+
+    sampler = ClockSampler(torch.cuda.current_device() if ws == 1 else local)
+    sampler.start()
+    time.sleep(0.3)
+    r = time_workload(S, spec, device, args.steps, args.warmup, rank, ws)
+    clocks = sampler.summary(r["t0"], r["t1"])
+    sampler.stop()
+
+    ms = r["total_ms"] / args.steps
+    launch_avg = sum(r["launch_ms"]) / len(r["launch_ms"])
+    # max over ranks
+    if ws > 1:
+        t = torch.tensor([ms, launch_avg], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, launch_avg = float(t[0]), float(t[1])
+    flops = spec.flops()
+    value = ws * flops / (ms * 1e-3) / 1e12
+
+    e2e_ms, h2d, d2h = time_e2e(S, spec, device, max(3, min(args.steps, 20)), 2)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e = ws * flops / (e2e_ms * 1e-3) / 1e12
+
+    per_config = {}
+    if args.per_config and rank == 0:
+        for name, sp in W.SPECS.items():
+            if name == spec.name:
+                continue
+            rr = time_workload(S, sp, device, max(3, args.steps // 4), 3, 0, 1)
+            lm = sum(rr["launch_ms"]) / len(rr["launch_ms"])
+            per_config[name] = dict(ms=lm, tflops=sp.flops() / (lm * 1e-3) / 1e12,
+                                    gbs=sp.bytes() / (lm * 1e-3) / 1e9)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(spec, budget_s=args.cpu_budget)
+        cpu.pop("seconds", None)
+
+    achieved = flops / (launch_avg * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    khash = kernel_source_hash()
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt2 q,k,v; rel-pos tables N(0,0.02^2))",
+        "config": {"workload": spec.name, "B": spec.B, "H": spec.Hq, "T": spec.Tq, "head_dim": spec.d,
+                   "grid": list(spec.q_hw) if spec.q_hw else None, "bias": "decomposed rel-pos",
+                   "l2": f"{r['nsets']} rotating input sets of {r['set_bytes'] / 1e6:.1f} MB (> L2)",
+                   "parallelism": f"replica x{ws} (independent problems per GPU)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                     "traffic": ncu_traffic(khash, spec.name),
+                     "flops_per_launch": flops, "launch_ms": launch_avg,
+                     "frac_of_spec_2250": achieved / 2250.0},
+        "e2e": {"value": e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "cpu_baseline": cpu,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "kernel_source_hash": khash,
+    }
+    if per_config:
+        line["per_config"] = per_config
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    spec = W.SPECS[args.workload]
+    vals = []
+    info = None
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        info = cpu_oracle_sample(spec, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(info["value"])
+    value = sum(vals) / len(vals)
+    secs = info.pop("seconds")
+    info["value"] = value
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "B": spec.B, "H": spec.Hq, "T": spec.Tq, "head_dim": spec.d},
+        "cpu_baseline": info,
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="sam_global", choices=sorted(W.SPECS))
+    ap.add_argument("--per-config", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * libsdpa -- fused scaled-dot-product-attention forward for NVIDIA B200 (sm_100a).
+ *
+ * Computes, for every batch b, query head h and query row i,
+ *
+ *     out[b,h,i,:] = softmax_j( scale * q[b,h,i,:] . k[b,hk,j,:] + bias[i,j] + mask[b,h,i,j] ) . v[b,hk,j,:]
+ *
+ * (Axon PR "Add scaled_dot_product_attention", description: softmax(Q.K^T*scale
+ * + mask).V over rank-4 inputs), where
+ *
+ *   - hk = h / (Hq / Hkv): grouped-query / multi-query attention by repeating
+ *     each key/value head Hq/Hkv times consecutively (Axon PR, GQA/MQA item);
+ *   - bias is the decomposed relative-position term of the SAM image encoder,
+ *     computed from the UNSCALED query inside the kernel, never materialised
+ *     (mlx-examples issue "segment_anything: fuse attention with
+ *     mx.fast.scaled_dot_product_attention": add_decomposed_rel_pos added to
+ *     (q*scale)@k^T before the softmax, and the point of fusing is not to
+ *     build the T_q x T_kv matrix; candle PR "SDPA with Relative Positional
+ *     Embeddings": term_h / term_w injected into the scores):
+ *         bias[i,j] = q_i . Rh[qh(i) - kh(j) + Kh - 1] + q_i . Rw[qw(i) - kw(j) + Kw - 1]
+ *         qh(i) = i / q_hw[1], qw(i) = i % q_hw[1], kh(j) = j / k_hw[1], kw(j) = j % k_hw[1],
+ *         Kh = k_hw[0], Kw = k_hw[1];
+ *   - mask is one of the Axon :mask forms (Axon PR, :mask option) -- causal
+ *     with an offset, a sliding window with an offset, or a runtime additive
+ *     float / boolean tensor broadcast to [B, Hq, Tq, Tkv] (mlx issue: the
+ *     mask argument is an arbitrary additive array).
+ *
+ * Layout: every tensor is dense row-major "bhsd": q and out [B, Hq, Tq, d],
+ * k and v [B, Hkv, Tkv, d], in the I/O dtype.  All data pointers are DEVICE
+ * pointers owned by the caller; the library keeps no reference after a call
+ * returns (it caches only TMA descriptors and a scratch buffer, see below).
+ *
+ * Every entry point is asynchronous on `stream` (no host synchronisation)
+ * unless stated otherwise, and returns SDPA_OK (0) or a negative sdpa_status.
+ * Argument errors are detected on the host before anything is launched.
+ */
+#ifndef SDPA_H_
+#define SDPA_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* I/O element type.  F32 runs on the exact CUDA-core path (no TF32: the fp32
+   tolerance of 1e-4 is below TF32's 10-bit mantissa); BF16 accumulates in fp32
+   and rounds the output to nearest-even. */
+typedef enum { SDPA_F32 = 0, SDPA_BF16 = 1 } sdpa_dtype_t;
+
+/* Mask kinds (Axon PR, :mask option).  Readings of what the pages leave open:
+   CAUSAL   key j visible from row i iff j <= i + offset.
+   SLIDING  visible iff i + offset - window < j <= i + offset (window keys,
+            diagonal included; one-sided, i.e. causal within the window).
+   ADD_FLOAT  additive tensor in the I/O dtype (-inf allowed).
+   BOOL     uint8 tensor, nonzero = attend, zero = excluded.
+   A row that sees no key produces a zero output row (and lse = -inf). */
+typedef enum {
+  SDPA_MASK_NONE = 0,
+  SDPA_MASK_CAUSAL = 1,
+  SDPA_MASK_SLIDING = 2,
+  SDPA_MASK_ADD_FLOAT = 3,
+  SDPA_MASK_BOOL = 4
+} sdpa_mask_kind_t;
+
+/* Host-side mask description; `mask_ptr` arguments point to one of these.
+   It may be NULL for NONE and for CAUSAL with offset 0.
+   For ADD_FLOAT / BOOL, element (b, h, i, j) is read at
+   data[b*stride_b + h*stride_h + i*stride_q + j] (element strides; a stride of
+   0 broadcasts that axis; the key axis is contiguous). */
+typedef struct {
+  int64_t offset;     /* CAUSAL / SLIDING diagonal offset (default 0)      */
+  int64_t window;     /* SLIDING window w >= 1                              */
+  const void* data;   /* device pointer, ADD_FLOAT (I/O dtype) or BOOL (u8) */
+  int64_t stride_b;
+  int64_t stride_h;
+  int64_t stride_q;
+} sdpa_mask_t;
+
+typedef enum {
+  SDPA_OK = 0,
+  SDPA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, Hq % Hkv != 0, aliasing, ... */
+  SDPA_ERR_UNSUPPORTED = -2,  /* legal request this build does not implement (d not in
+                                 {16,64,128}, rel-pos with q_hw != k_hw, path forced
+                                 onto a kernel that cannot take the problem) */
+  SDPA_ERR_MISALIGNED = -3,   /* a pointer or stride breaks the 16-byte rule of the
+                                 forced tensor-core path */
+  SDPA_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (launch, copy) */
+  SDPA_ERR_TIMEOUT = -5,      /* a device-side bounded wait expired (see
+                                 sdpa_last_device_error) */
+  SDPA_ERR_CAPACITY = -6      /* the request exceeds a fixed-size buffer of this entry point */
+} sdpa_status;
+
+/* Kernel families.  AUTO picks per shape; the others force one family and
+   return SDPA_ERR_UNSUPPORTED when it cannot take the problem. */
+typedef enum {
+  SDPA_PATH_AUTO = 0,
+  SDPA_PATH_EXACT = 1,     /* CUDA-core FFMA online softmax; every feature, fp32 and bf16 */
+  SDPA_PATH_TCGEN05 = 2,   /* TMA + tcgen05/TMEM flash kernel; bf16, d in {64,128} */
+  SDPA_PATH_SMALL_D = 3,   /* packed d=16 kernel, one query row per thread; bf16 */
+  SDPA_PATH_SPLIT_KV = 4   /* split-KV with in-kernel merge, short Tq / long Tkv; bf16, d=16..128 */
+} sdpa_path_t;
+
+/*
+ * sdpa_fwd -- the fused forward.
+ *   q, k, v, out : device pointers (layout above).  out must not overlap q, k
+ *                  or v.  k and v may be NULL only when Tkv == 0; q and out
+ *                  only when B*Hq*Tq == 0.
+ *   dtype        : sdpa_dtype_t of q, k, v, out, the rel-pos tables and an
+ *                  ADD_FLOAT mask.
+ *   B, Hq, Hkv, Tq, Tkv : B >= 0, Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
+ *                  Tq >= 0, Tkv >= 0.
+ *   d            : head_dim, one of 16, 64, 128.
+ *   scale        : score scale, finite (the Axon default 1/sqrt(d) is applied
+ *                  by the Python binding, not here).
+ *   mask_kind, mask_ptr : sdpa_mask_kind_t and a host sdpa_mask_t* (see above).
+ *   rel_pos_h, rel_pos_w : device tables [2*k_hw[0]-1, d] and [2*k_hw[1]-1, d]
+ *                  in the I/O dtype, shared by every batch and head; both NULL
+ *                  disables the bias, exactly one NULL is INVALID_ARG.
+ *   q_hw, k_hw   : host int[2] patch grids (height, width) with
+ *                  q_hw[0]*q_hw[1] == Tq and k_hw[0]*k_hw[1] == Tkv; required
+ *                  with rel-pos, ignored otherwise.  q_hw != k_hw is
+ *                  UNSUPPORTED (the pages give the equal-size formula only).
+ *   stream       : CUDA stream the work is enqueued on.
+ */
+int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+             int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
+             int mask_kind, const void* mask_ptr,
+             const void* rel_pos_h, const void* rel_pos_w,
+             const int* q_hw, const int* k_hw,
+             cudaStream_t stream);
+
+/*
+ * sdpa_fwd_ex -- sdpa_fwd plus two options.
+ *   lse  : NULL, or a device float [B, Hq, Tq] receiving the natural-log
+ *          sum-exp of each score row (m + log l; -inf for a row with no
+ *          visible key).
+ *   path : sdpa_path_t; AUTO behaves like sdpa_fwd.
+ * The split-KV path keeps its partial results in a scratch buffer that the
+ * library allocates on first use per device and grows when needed (never
+ * freed until exit); calls on one device that overlap on the GPU must not use
+ * that path concurrently.
+ */
+int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
+                int mask_kind, const void* mask_ptr,
+                const void* rel_pos_h, const void* rel_pos_w,
+                const int* q_hw, const int* k_hw,
+                float* lse, int path, cudaStream_t stream);
+
+/* The path AUTO would take for this problem (a non-negative sdpa_path_t), or a
+   negative sdpa_status when the arguments are invalid.  Launches nothing;
+   pointers are only checked for NULL and alignment. */
+int sdpa_select_path(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                     int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                     int mask_kind, const void* mask_ptr,
+                     const void* rel_pos_h, const void* rel_pos_w,
+                     const int* q_hw, const int* k_hw);
+
+/*
+ * sdpa_fwd_host -- the same forward on HOST buffers.  Copies q, k, v, the
+ * rel-pos tables and an ADD_FLOAT/BOOL mask (its data pointer is then a HOST
+ * pointer, read with the strides given) to device buffers the library keeps
+ * per device (grown as needed), runs sdpa_fwd_ex on `stream`, copies the
+ * result into the host buffer `out` and synchronises `stream` before
+ * returning.  For transfer speed the host buffers should be pinned.  Not
+ * reentrant across host threads on the same device.
+ */
+int sdpa_fwd_host(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                  int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
+                  int mask_kind, const void* mask_ptr,
+                  const void* rel_pos_h, const void* rel_pos_w,
+                  const int* q_hw, const int* k_hw,
+                  int path, cudaStream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device error word of the
+   current device: SDPA_OK, or SDPA_ERR_TIMEOUT when a kernel gave up a bounded
+   wait since the last call (its output is then undefined), or SDPA_ERR_CUDA
+   when the synchronisation itself failed. */
+int sdpa_last_device_error(cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char* sdpa_strerror(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sdpa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_H_ */

@@ -156,14 +156,22 @@ int oracle_sdpa_rows(const double* q, const double* k, const double* v,
 #else
           const long long idx = qh - a + k_h - 1;
 #endif
+#if ORACLE_PLANT == 3
+          relh[a] = dot(qi, th + (idx % (2 * k_w - 1)) * d, d); /* swapped tables differ in size */
+#else
           relh[a] = dot(qi, th + idx * d, d);
+#endif
         }
         for (int a = 0; a < k_w; ++a) {
           const long long idx = qw - a + k_w - 1;
 #if ORACLE_PLANT == 2
           relw[a] = 0.0;
 #else
+#if ORACLE_PLANT == 3
+          relw[a] = dot(qi, tw + (idx % (2 * k_h - 1)) * d, d);
+#else
           relw[a] = dot(qi, tw + idx * d, d);
+#endif
 #endif
         }
       }

@@ -1,0 +1,121 @@
+"""The C-ABI library loads, exports every symbol include/sdpa.h declares, and
+rejects bad arguments on the host before touching a GPU (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_sdpa_fwd_b200 as S
+from attention_sdpa_fwd_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w[\w\s\*]*?\b(sdpa_\w+)\s*\(", txt, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return S.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "sdpa_fwd" in names and "sdpa_fwd_ex" in names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert set(names) <= set(S.EXPORTS) | set(names)
+    assert set(S.EXPORTS) <= set(names), "binding lists a symbol the header does not declare"
+
+
+def test_version_and_strerror(L):
+    assert S.sdpa_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert S.sdpa_strerror(code) not in ("", "unknown status")
+    assert S.sdpa_strerror(12345) == "unknown status"
+
+
+# Distinct fake device addresses (never dereferenced: validation fails first).
+Q, K, V, O = 0x100000, 0x200000, 0x300000, 0x400000
+BF16 = S.SDPA_BF16
+
+
+def sel(*a, **kw):
+    args = dict(q=Q, k=K, v=V, out=O, dtype=BF16, B=1, Hq=4, Hkv=2, Tq=8, Tkv=8, d=64,
+                mask_kind=0, mask=None, rh=None, rw=None, q_hw=None, k_hw=None)
+    args.update(kw)
+    m = args["mask"]
+    return S.sdpa_select_path(args["q"], args["k"], args["v"], args["out"], args["dtype"], args["B"],
+                              args["Hq"], args["Hkv"], args["Tq"], args["Tkv"], args["d"], args["mask_kind"],
+                              ctypes.byref(m) if m is not None else None, args["rh"], args["rw"],
+                              args["q_hw"], args["k_hw"])
+
+
+def test_valid_problem_selects_a_path(L):
+    assert sel() >= 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), -1),                 # Hq % Hkv != 0
+    (dict(Hkv=0), -1),
+    (dict(B=-1), -1),
+    (dict(Tq=-5), -1),
+    (dict(d=32), -2),                        # head_dim outside {16, 64, 128}
+    (dict(d=96), -2),
+    (dict(dtype=7), -1),
+    (dict(q=0), -1),                         # NULL q with work to do
+    (dict(k=0), -1),
+    (dict(out=0), -1),
+    (dict(out=Q + 64), -1),                  # out overlaps q
+    (dict(q=Q + 1), -3),                     # bf16 pointer not 2-byte aligned
+    (dict(mask_kind=9), -1),
+    (dict(mask_kind=S.MASK_SLIDING), -1),    # sliding needs a descriptor
+    (dict(mask_kind=S.MASK_SLIDING, mask=S.sdpa_mask_t(window=0)), -1),
+    (dict(mask_kind=S.MASK_FLOAT), -1),      # float mask needs a descriptor
+    (dict(mask_kind=S.MASK_FLOAT, mask=S.sdpa_mask_t(data=None)), -1),
+    (dict(mask_kind=S.MASK_FLOAT, mask=S.sdpa_mask_t(data=0x500001, stride_q=8)), -3),
+    (dict(mask_kind=S.MASK_BOOL, mask=S.sdpa_mask_t(data=0x500000, stride_q=-8)), -1),
+    (dict(rh=0x600000), -1),                 # only one table
+    (dict(rh=0x600000, rw=0x700000), -1),    # tables without grids
+    (dict(rh=0x600000, rw=0x700000, q_hw=(2, 3), k_hw=(2, 4)), -1),   # grid != Tq
+    (dict(rh=0x600000, rw=0x700000, q_hw=(2, 4), k_hw=(4, 2)), -2),   # q_hw != k_hw
+    (dict(rh=0x600000, rw=0x700000, q_hw=(0, 8), k_hw=(0, 8)), -1),
+    (dict(rh=0x600001, rw=0x700000, q_hw=(2, 4), k_hw=(2, 4)), -3),
+])
+def test_invalid_arguments_rejected(L, kw, code):
+    assert sel(**kw) == code
+
+
+def test_empty_problems_are_valid(L):
+    assert sel(B=0, q=0, out=0) >= 0
+    assert sel(Tq=0, q=0, out=0) >= 0
+    assert sel(Tkv=0, k=0, v=0) >= 0
+
+
+def test_forward_rejects_before_launch(L):
+    # invalid problems return their status from sdpa_fwd / sdpa_fwd_ex without touching a device
+    rc = S.sdpa_fwd(Q, K, V, O, BF16, 1, 3, 2, 8, 8, 64, 0.125, 0, None, None, None, None, None, None)
+    assert rc == -1
+    rc = S.sdpa_fwd_ex(Q, K, V, O, BF16, 1, 4, 2, 8, 8, 64, float("nan"), 0, None, None, None, None, None,
+                       None, 0, None)
+    assert rc == -1
+    rc = S.sdpa_fwd_ex(Q, K, V, O, BF16, 1, 4, 2, 8, 8, 64, 0.1, 0, None, None, None, None, None, None, 17, None)
+    assert rc == -1
+    rc = S.sdpa_fwd_host(Q, K, V, O, BF16, 1, 4, 2, 8, 8, 32, 0.1, 0, None, None, None, None, None, 0, None)
+    assert rc == -2
+
+
+def test_binding_has_no_cpu_path():
+    import torch
+    q = torch.zeros(1, 1, 4, 16)
+    with pytest.raises(ValueError):
+        S.sdpa(q, q, q)

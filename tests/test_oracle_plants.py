@@ -30,6 +30,6 @@ def test_planted_mistake_is_caught(plant, tmp_path):
     for pin in ALL_PINS:
         try:
             pin(lib)
-        except AssertionError:
+        except Exception:  # an assertion, or a planted copy rejecting its inputs
             failed.append(pin.__name__)
     assert failed, f"no pin caught planted mistake {plant}: {PLANTS[plant]}"
