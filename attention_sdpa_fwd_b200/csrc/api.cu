@@ -123,7 +123,7 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
 }
 
 int choose_path(const Problem& pr) {
-  (void)pr;
+  if (tc_check(pr.p, pr.dtype) == SDPA_OK) return SDPA_PATH_TCGEN05;
   return SDPA_PATH_EXACT;
 }
 
@@ -136,7 +136,12 @@ int run(const Problem& pr, int path, cudaStream_t stream) {
   cudaError_t e;
   switch (path) {
     case SDPA_PATH_EXACT: e = launch_exact(p, pr.dtype, stream); break;
-    case SDPA_PATH_TCGEN05:
+    case SDPA_PATH_TCGEN05: {
+      const int rc = tc_check(p, pr.dtype);
+      if (rc != SDPA_OK) return rc;
+      e = launch_tc(p, stream);
+      break;
+    }
     case SDPA_PATH_SMALL_D:
     case SDPA_PATH_SPLIT_KV: return SDPA_ERR_UNSUPPORTED;
     default: return SDPA_ERR_INVALID_ARG;

@@ -60,5 +60,7 @@ __host__ __device__ __forceinline__ void key_range(const Params& p, long long i,
 
 // Launchers (one per kernel family); each returns a cudaError_t of the launch.
 cudaError_t launch_exact(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
+int tc_check(const Params& p, sdpa_dtype_t dtype);  // SDPA_OK or why the tensor-core kernel cannot run
+cudaError_t launch_tc(const Params& p, cudaStream_t stream);
 
 }  // namespace sdpa

@@ -1,0 +1,645 @@
+// Tensor-core fused SDPA forward for sm_100a: TMA + tcgen05/TMEM, online
+// softmax, in-kernel decomposed rel-pos bias and masks.
+//
+// softmax(Q.K^T*scale + bias).V without materialising the T_q x T_kv score
+// matrix (mlx-examples issue "segment_anything: fuse attention with
+// mx.fast.scaled_dot_product_attention": the fused call avoids the 4096x4096
+// per-head matrix and the separate softmax pass).  The bias is SAM's
+// decomposed relative position (candle PR "SDPA with Relative Positional
+// Embeddings": term_h / term_w injected into the scores) or an Axon :mask
+// (Axon PR "Add scaled_dot_product_attention", :mask option).
+//
+// One CTA owns 256 query rows of one (batch, head) as two 128-row tiles A/B
+// and streams the K/V tiles of its kv head (hk = h / (Hq/Hkv), Axon PR GQA
+// item) through a shared-memory ring.  Warp roles (384 threads):
+//   warps 0-3   softmax of tile A (thread = query row = TMEM lane)
+//   warps 4-7   softmax of tile B
+//   warp  8     TMA producer (Q once, then K_j / V_j per stage)
+//   warp  9     TMEM owner and MMA issuer (one elected thread)
+//   warps 10-11 idle
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D, 256+2D).
+// P (bf16) overwrites the first BN/2 columns of its S tile and is the A
+// operand of the P.V MMA straight from TMEM.
+//
+// Per KV tile j the MMA warp issues S_t = Q_t.K_j^T (SS, both K-major) and,
+// once softmax t has written P_t, O_t += P_t.V_j (TS, V MN-major).  The commit
+// that signals "S_t(j+1) ready" also covers O_t += P_t(j).V_j, so softmax t may
+// rescale O_t in place when its running max grows.  It does so only when the
+// max grows by more than 2^8: every term stays relative to the same (stale)
+// max, so the final O/l is unchanged up to rounding.
+//
+// Rel-pos: before the loop, Ph_t = Q_t.Rh^T and Pw_t = Q_t.Rw^T are computed
+// on the tensor cores into TMEM (tables zero-padded to a multiple of 16
+// rows), and each thread scatters its row's rel_h[i, kh] = Ph[i, qh - kh + Kh - 1]
+// and rel_w[i, kw] = Pw[i, qw - kw + Kw - 1] (times log2 e) into shared
+// memory, from where the loop adds them to the scores before the row max.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace sdpa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kRowsPerTile = 128;
+constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-pos path
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3 };
+
+struct TcArgs {
+  CUtensorMap tq, tk, tv, trh, trw;
+  void* out;
+  float* lse;
+  const void* mask;
+  long long msb, msh, msq;
+  long long offset, window;
+  int B, Hq, Hkv, Tq, Tkv, group;
+  int mask_kind;
+  float scale_log2;
+  int qw_n, kh_n, kw_n;
+  int rel_n;  // rows of the padded rel tables (multiple of 16, <= 128)
+  int* err;
+};
+
+template <int D, int BN, int KW, int NS>
+struct Layout {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kQBytes = kPanels * kRowsPerTile * 128;  // one Q tile
+  static constexpr int kKVBytes = kPanels * BN * 128;           // one K or V tile
+  static constexpr int kRelRows = KW > 0 ? kRelHMax + KW : 0;   // rel_h rows then rel_w rows, 256 floats each
+  static constexpr int oQ = 0;
+  static constexpr int oK = oQ + 2 * kQBytes;
+  static constexpr int oV = oK + NS * kKVBytes;
+  static constexpr int oRel = oV + NS * kKVBytes;
+  static constexpr int oBar = oRel + kRelRows * 256 * 4;
+  static constexpr int kBars = 3 * NS + 10;
+  static constexpr int kTotal = oBar + kBars * 8 + 16;
+  static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "shared memory budget");
+  static_assert(KW == 0 || (BN % (KW > 0 ? KW : 1) == 0), "key tile must hold whole key-grid rows");
+};
+
+template <int D, int BN, int KW, int MASK, int NS>
+__global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constant__ TcArgs args) {
+  using L = Layout<D, BN, KW, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + L::oQ;
+  uint8_t* sK = smem + L::oK;
+  uint8_t* sV = smem + L::oV;
+  float* sRel = reinterpret_cast<float*>(smem + L::oRel);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::oBar);
+  uint64_t* k_full = bars;               // [NS]  TMA -> MMA
+  uint64_t* v_full = bars + NS;          // [NS]
+  uint64_t* kv_empty = bars + 2 * NS;    // [NS]  MMA commit -> TMA
+  uint64_t* q_full = bars + 3 * NS;      // Q tiles (and rel tables) landed
+  uint64_t* s_full = q_full + 1;         // [2]   MMA commit -> softmax t
+  uint64_t* p_full = q_full + 3;         // [2]   softmax t (128 arrivals) -> MMA
+  uint64_t* o_done = q_full + 5;         // [2]   final MMA commit -> softmax t epilogue
+  uint64_t* rel_mma = q_full + 7;        // rel projections in TMEM (MMA commit)
+  uint64_t* rel_read = q_full + 8;       // projections read by all 256 softmax threads
+  uint64_t* fin = q_full + 9;            // last commit before TMEM release
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + L::kBars);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int qblk = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int hk = h / args.group;
+  const int q0 = qblk * 2 * kRowsPerTile;
+
+  // Key-tile range of this CTA (causal / sliding skip whole tiles).
+  int j_begin = 0, j_end = (args.Tkv + BN - 1) / BN;
+  if (MASK == TC_RANGE) {
+    const long long first = q0;
+    const long long last = (long long)min(q0 + 2 * kRowsPerTile, args.Tq) - 1;
+    long long lo = 0, hi = args.Tkv;
+    if (last + args.offset + 1 < hi) hi = last + args.offset + 1;
+    if (args.mask_kind == SDPA_MASK_SLIDING) lo = max(0LL, first + args.offset - args.window + 1);
+    if (hi <= lo) {
+      j_begin = j_end = 0;
+    } else {
+      j_begin = (int)(lo / BN);
+      j_end = (int)((hi + BN - 1) / BN);
+    }
+  }
+  const int n_tiles = j_end - j_begin;
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < L::kBars; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&p_full[0], kRowsPerTile);
+    mbar_init(&p_full[1], kRowsPerTile);
+    mbar_init(rel_read, 2 * kRowsPerTile);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  volatile int* abort_v = abort_flag;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&args.tq);
+      tma_prefetch_desc(&args.tk);
+      tma_prefetch_desc(&args.tv);
+      const int zq = b * args.Hq + h;
+      const int zk = b * args.Hkv + hk;
+      uint32_t qbytes = 2 * L::kQBytes;
+      if (KW > 0) qbytes += 2 * args.rel_n * 128;
+      mbar_expect_tx(q_full, qbytes);
+      for (int t = 0; t < 2; ++t)
+        for (int p = 0; p < L::kPanels; ++p)
+          tma_load_3d(sQ + t * L::kQBytes + p * kRowsPerTile * 128, &args.tq, q_full, p * 64,
+                      q0 + t * kRowsPerTile, zq);
+      if (KW > 0) {
+        // the rel tables borrow the last stage's K/V buffers until the projections are done
+        tma_load_3d(sK + (NS - 1) * L::kKVBytes, &args.trh, q_full, 0, 0, 0);
+        tma_load_3d(sV + (NS - 1) * L::kKVBytes, &args.trw, q_full, 0, 0, 0);
+      }
+      bool ok = true;
+      int issued = 0;
+      for (int jj = 0; jj < n_tiles && ok; ++jj) {
+        const int s = jj % NS;
+        const int use = jj / NS;
+        if (use > 0) ok = mbar_wait(&kv_empty[s], (use - 1) & 1, abort_v, args.err);
+        if (ok && KW > 0 && jj == NS - 1) ok = mbar_wait(rel_mma, 0, abort_v, args.err);
+        if (!ok) break;
+        const int key0 = (j_begin + jj) * BN;
+        mbar_expect_tx(&k_full[s], L::kKVBytes);
+        for (int p = 0; p < L::kPanels; ++p)
+          tma_load_3d(sK + s * L::kKVBytes + p * BN * 128, &args.tk, &k_full[s], p * 64, key0, zk);
+        mbar_expect_tx(&v_full[s], L::kKVBytes);
+        for (int p = 0; p < L::kPanels; ++p)
+          tma_load_3d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, zk);
+        issued = jj + 1;
+      }
+      if (!ok) {
+        // abandoned: let the copies already in flight land before the CTA exits
+        mbar_wait(q_full, 0, nullptr, args.err);
+        for (int jj = max(0, issued - NS); jj < issued; ++jj) {
+          mbar_wait(&k_full[jj % NS], (jj / NS) & 1, nullptr, args.err);
+          mbar_wait(&v_full[jj % NS], (jj / NS) & 1, nullptr, args.err);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t id_qk = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, D, false, true);
+      const uint32_t sq = smem_u32(sQ), sk = smem_u32(sK), sv = smem_u32(sV);
+      bool ok = mbar_wait(q_full, 0, abort_v, args.err);
+      auto qk = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          const uint32_t a = sq + t * L::kQBytes + (kk >> 2) * (kRowsPerTile * 128) + koff;
+          const uint32_t bb = sk + s * L::kKVBytes + (kk >> 2) * (BN * 128) + koff;
+          mma_ss(tbase + t * 128, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id_qk, kk > 0);
+        }
+      };
+      auto pv = [&](int t, int s, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t bb = sv + s * L::kKVBytes + kk * 16 * 128;
+          mma_ts(tbase + 256 + t * D, tbase + t * 128 + kk * 8, sdesc_sw128(bb, BN * 128, 1024), id_pv,
+                 (!first) || kk > 0);
+        }
+      };
+      if (ok && KW > 0) {
+        // rel projections: Ph_t -> cols [256t, 256t+rel_n), Pw_t -> [256t+128, 256t+128+rel_n)
+        const uint32_t id_rel = idesc_bf16_f32(128, args.rel_n, false, false);
+        const uint32_t rh = sk + (NS - 1) * L::kKVBytes, rw = sv + (NS - 1) * L::kKVBytes;
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          for (int w = 0; w < 2; ++w)
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t a = sq + t * L::kQBytes + kk * 32;
+              const uint32_t bb = (w == 0 ? rh : rw) + kk * 32;
+              mma_ss(tbase + t * 256 + w * 128, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id_rel,
+                     kk > 0);
+            }
+        mma_commit(rel_mma);
+        ok = mbar_wait(rel_read, 0, abort_v, args.err);
+      }
+      // prologue: S_A(0), S_B(0)
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_v, args.err);
+      if (ok) {
+        tc_fence_after();
+        qk(0, 0);
+        mma_commit(&s_full[0]);
+        qk(1, 0);
+        mma_commit(&s_full[1]);
+      }
+      for (int jj = 0; jj < n_tiles && ok; ++jj) {
+        const int s = jj % NS;
+        ok = mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err);
+        if (!ok) break;
+        // tile A: O_A += P_A V_j, then S_A(j+1)
+        ok = mbar_wait(&p_full[0], jj & 1, abort_v, args.err);
+        if (!ok) break;
+        tc_fence_after();
+        pv(0, s, jj == 0);
+        const bool more = jj + 1 < n_tiles;
+        const int s1 = (jj + 1) % NS;
+        if (more) {
+          ok = mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          qk(0, s1);
+          mma_commit(&s_full[0]);
+        }
+        // tile B: O_B += P_B V_j, release stage j, then S_B(j+1)
+        ok = mbar_wait(&p_full[1], jj & 1, abort_v, args.err);
+        if (!ok) break;
+        tc_fence_after();
+        pv(1, s, jj == 0);
+        mma_commit(&kv_empty[s]);
+        if (more) {
+          qk(1, s1);
+          mma_commit(&s_full[1]);
+        }
+      }
+      mma_commit(&o_done[0]);
+      mma_commit(&o_done[1]);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax of tile t
+    const int t = warp >> 2;
+    const int lr = (warp & 3) * 32 + lane;   // row within the tile = TMEM lane
+    const int row = t * kRowsPerTile + lr;   // row within the CTA
+    const long long qi = (long long)q0 + row;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tbase + lane_off + t * 128;
+    const uint32_t o_addr = tbase + lane_off + 256 + t * D;
+    bool ok = true;
+    float* relh_s = sRel;                  // [kRelHMax][256]
+    float* relw_s = sRel + kRelHMax * 256;  // [KW][256]
+
+    if constexpr (KW > 0) if (n_tiles > 0) {
+      // scatter this row's rel_h / rel_w (log2 e prescaled) into shared memory
+      ok = __all_sync(0xffffffffu, mbar_wait(rel_mma, 0, abort_v, args.err));
+      tc_fence_after();
+      const int qw_n = args.qw_n, kh_n = args.kh_n;
+      const int qh = (int)(qi / qw_n), qw = (int)(qi % qw_n);
+      if (ok) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int base_idx = w == 0 ? qh + kh_n - 1 : qw + KW - 1;
+          const int nk = w == 0 ? kh_n : KW;
+          float* dst = w == 0 ? relh_s : relw_s;
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            if (c0 < args.rel_n) {
+              uint32_t r[32];
+              tmem_ld32(tbase + lane_off + t * 256 + w * 128 + c0, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int k = base_idx - (c0 + i);  // key-grid coordinate reached through table row c0+i
+                if (k >= 0 && k < nk) dst[k * 256 + row] = __uint_as_float(r[i]) * kLog2e;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(rel_read);
+    }
+
+    // per-row visible key range (causal / sliding)
+    long long lo_i = 0, hi_i = args.Tkv;
+    if constexpr (MASK == TC_RANGE) {
+      if (qi + args.offset + 1 < hi_i) hi_i = qi + args.offset + 1;
+      if (args.mask_kind == SDPA_MASK_SLIDING) lo_i = max(0LL, qi + args.offset - args.window + 1);
+    }
+    const bool row_valid = qi < args.Tq;
+    const long long mrow = (long long)b * args.msb + (long long)h * args.msh + qi * args.msq;
+
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int jj = 0; jj < n_tiles && ok; ++jj) {
+      const int j0 = (j_begin + jj) * BN;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], jj & 1, abort_v, args.err));
+      if (!ok) break;
+      tc_fence_after();
+      float x[BN];
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        if (c0 + 32 <= BN) {
+          uint32_t r[32];
+          tmem_ld32(s_addr + c0, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[c0 + i] = __uint_as_float(r[i]);
+        } else {
+          uint32_t r[16];
+          tmem_ld16(s_addr + c0, r);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[c0 + i] = __uint_as_float(r[i]);
+        }
+      }
+      tmem_wait_ld();
+
+      // scale (and rel-pos bias), in log2 units
+      if constexpr (KW > 0) {
+        const int kh0 = j0 / KW;
+#pragma unroll
+        for (int g = 0; g < BN / KW; ++g) {
+          const int khi = kh0 + g;
+          const float rh = khi < args.kh_n ? relh_s[khi * 256 + row] : 0.f;
+#pragma unroll
+          for (int c = 0; c < KW; ++c)
+            x[g * KW + c] = fmaf(x[g * KW + c], args.scale_log2, relw_s[c * 256 + row] + rh);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) x[c] *= args.scale_log2;
+      }
+      if constexpr (MASK == TC_RANGE) {
+        if (!(j0 >= lo_i && j0 + BN <= hi_i)) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (j0 + c < lo_i || j0 + c >= hi_i) x[c] = -INFINITY;
+        }
+      } else if constexpr (MASK == TC_FLOAT) {
+        if (row_valid) {
+        const __nv_bfloat16* mp = static_cast<const __nv_bfloat16*>(args.mask) + mrow + j0;
+        if (j0 + BN <= args.Tkv) {
+#pragma unroll
+          for (int c = 0; c < BN; c += 8) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(mp + c));
+            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[c + u] = fmaf(__bfloat162float(e[u]), kLog2e, x[c + u]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (j0 + c < args.Tkv) x[c] = fmaf(__bfloat162float(mp[c]), kLog2e, x[c]);
+        }
+        }
+      } else if constexpr (MASK == TC_BOOL) {
+        if (row_valid) {
+        const uint8_t* mp = static_cast<const uint8_t*>(args.mask) + mrow + j0;
+        if (j0 + BN <= args.Tkv) {
+#pragma unroll
+          for (int c = 0; c < BN; c += 16) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(mp + c));
+            const uint8_t* e = reinterpret_cast<const uint8_t*>(&raw);
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              if (e[u] == 0) x[c + u] = -INFINITY;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (j0 + c < args.Tkv && mp[c] == 0) x[c] = -INFINITY;
+        }
+        }
+      }
+      if (j0 + BN > args.Tkv) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (j0 + c >= args.Tkv) x[c] = -INFINITY;
+      }
+
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m_run, mx);
+      const bool need = m_new > m_run + kRescaleThreshold;  // false while both are -inf
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_run - m_new);  // 0 when m_run == -inf
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      if (jj > 0 && __any_sync(0xffffffffu, need)) {
+        // O_t row *= alpha (warp-collective; alpha is 1 where the max did not move)
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(o_addr + c0, r);
+        }
+      }
+
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      float rowsum = 0.f;
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2_approx(x[c] - m_use);
+        const float p1 = ex2_approx(x[c + 1] - m_use);
+        rowsum += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l_run += rowsum;
+#pragma unroll
+      for (int c0 = 0; c0 < BN / 2; c0 += 8) {
+        uint32_t r8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r8[i] = pk[c0 + i];
+        tmem_st8(s_addr + c0, r8);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // epilogue: O / l -> bf16, rows past Tq are not stored
+    const long long zq = (long long)b * args.Hq + h;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (zq * args.Tq + qi) * D;
+    if (n_tiles == 0) {
+      if (row_valid) {
+#pragma unroll
+        for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+        if (args.lse) args.lse[zq * args.Tq + qi] = -INFINITY;
+      }
+    } else {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, abort_v, args.err));
+      tc_fence_after();
+      if (ok) {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c0, r);
+          tmem_wait_ld();
+          if (row_valid) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[c + 0]) * inv, __uint_as_float(r[c + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(r[c + 2]) * inv, __uint_as_float(r[c + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(r[c + 4]) * inv, __uint_as_float(r[c + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(r[c + 6]) * inv, __uint_as_float(r[c + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + c0 + c) = v;
+            }
+          }
+        }
+        if (row_valid && args.lse)
+          args.lse[zq * args.Tq + qi] = l_run > 0.f ? m_run * kLn2 + logf(l_run) : -INFINITY;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) {
+    if (lane == 0 && n_tiles > 0) {
+      // nothing this CTA issued may still be writing TMEM when it is released
+      mma_commit(fin);
+      mbar_wait(fin, 0, nullptr, args.err);
+    }
+    __syncwarp();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+template <int D, int BN, int KW, int MASK, int NS>
+cudaError_t launch_one(const TcArgs& a, dim3 grid, cudaStream_t stream) {
+  using L = Layout<D, BN, KW, NS>;
+  auto kern = flash_fwd_tc<D, BN, KW, MASK, NS>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int BN, int KW, int NS>
+cudaError_t dispatch_mask(int mk, const TcArgs& a, dim3 grid, cudaStream_t stream) {
+  switch (mk) {
+    case TC_NONE: return launch_one<D, BN, KW, TC_NONE, NS>(a, grid, stream);
+    case TC_RANGE: return launch_one<D, BN, KW, TC_RANGE, NS>(a, grid, stream);
+    case TC_FLOAT: return launch_one<D, BN, KW, TC_FLOAT, NS>(a, grid, stream);
+    case TC_BOOL: return launch_one<D, BN, KW, TC_BOOL, NS>(a, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int BN, int KW, int NS>
+cudaError_t dispatch_mask_rel(int mk, const TcArgs& a, dim3 grid, cudaStream_t stream) {
+  switch (mk) {
+    case TC_NONE: return launch_one<D, BN, KW, TC_NONE, NS>(a, grid, stream);
+    case TC_RANGE: return launch_one<D, BN, KW, TC_RANGE, NS>(a, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int tc_mask_code(const Params& p) {
+  switch (p.mask_kind) {
+    case SDPA_MASK_NONE: return TC_NONE;
+    case SDPA_MASK_CAUSAL:
+    case SDPA_MASK_SLIDING: return TC_RANGE;
+    case SDPA_MASK_ADD_FLOAT: return TC_FLOAT;
+    case SDPA_MASK_BOOL: return TC_BOOL;
+  }
+  return -1;
+}
+
+}  // namespace
+
+// Whether the tensor-core kernel takes this (already validated) problem;
+// SDPA_OK, SDPA_ERR_UNSUPPORTED or SDPA_ERR_MISALIGNED.
+int tc_check(const Params& p, sdpa_dtype_t dtype) {
+  if (dtype != SDPA_BF16) return SDPA_ERR_UNSUPPORTED;
+  if (p.d != 64 && p.d != 128) return SDPA_ERR_UNSUPPORTED;
+  if (p.Tkv < 1 || p.Tq < 1) return SDPA_ERR_UNSUPPORTED;
+  if (p.B > 65535 || p.Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+  if (!al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.out)) return SDPA_ERR_MISALIGNED;
+  if (p.use_rel) {
+    if (p.d != 64) return SDPA_ERR_UNSUPPORTED;
+    const int kw = p.kw_n;
+    if (!(kw == 14 || kw == 16 || kw == 32 || kw == 64)) return SDPA_ERR_UNSUPPORTED;
+    if (p.kh_n > kRelHMax) return SDPA_ERR_UNSUPPORTED;
+    // the padded tables borrow one K/V stage buffer: at most BN rows
+    const int kmax = p.kh_n > kw ? p.kh_n : kw;
+    if (((2 * kmax - 1) + 15) / 16 * 16 > (kw == 14 ? 112 : 128)) return SDPA_ERR_UNSUPPORTED;
+    if (p.mask_kind == SDPA_MASK_ADD_FLOAT || p.mask_kind == SDPA_MASK_BOOL) return SDPA_ERR_UNSUPPORTED;
+    if (!al16(p.rel_h) || !al16(p.rel_w)) return SDPA_ERR_MISALIGNED;
+  }
+  if (p.mask_kind == SDPA_MASK_ADD_FLOAT) {
+    if (!al16(p.mask) || (p.msb % 8) || (p.msh % 8) || (p.msq % 8)) return SDPA_ERR_MISALIGNED;
+  }
+  if (p.mask_kind == SDPA_MASK_BOOL) {
+    if (!al16(p.mask) || (p.msb % 16) || (p.msh % 16) || (p.msq % 16)) return SDPA_ERR_MISALIGNED;
+  }
+  return SDPA_OK;
+}
+
+cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t rowb = (uint64_t)p.d * 2;
+  const int BN = (p.use_rel && p.kw_n == 14) ? 112 : 128;
+  bool ok = make_tmap_3d(&a.tq, p.q, bf, 2, p.d, p.Tq, (uint64_t)p.B * p.Hq, rowb, rowb * p.Tq, 64, 128, true);
+  ok = ok && make_tmap_3d(&a.tk, p.k, bf, 2, p.d, p.Tkv, (uint64_t)p.B * p.Hkv, rowb, rowb * p.Tkv, 64, BN, true);
+  ok = ok && make_tmap_3d(&a.tv, p.v, bf, 2, p.d, p.Tkv, (uint64_t)p.B * p.Hkv, rowb, rowb * p.Tkv, 64, BN, true);
+  if (p.use_rel) {
+    const int kmax = p.kh_n > p.kw_n ? p.kh_n : p.kw_n;
+    a.rel_n = ((2 * kmax - 1) + 15) / 16 * 16;
+    const uint64_t nh = 2 * p.kh_n - 1, nw = 2 * p.kw_n - 1;
+    ok = ok && make_tmap_3d(&a.trh, p.rel_h, bf, 2, p.d, nh, 1, rowb, rowb * nh, 64, a.rel_n, true);
+    ok = ok && make_tmap_3d(&a.trw, p.rel_w, bf, 2, p.d, nw, 1, rowb, rowb * nw, 64, a.rel_n, true);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  a.out = p.out;
+  a.lse = p.lse;
+  a.mask = p.mask;
+  a.msb = p.msb; a.msh = p.msh; a.msq = p.msq;
+  a.offset = p.offset; a.window = p.window;
+  a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.Tq = p.Tq; a.Tkv = p.Tkv; a.group = p.group;
+  a.mask_kind = p.mask_kind;
+  a.scale_log2 = p.scale * kLog2e;
+  a.qw_n = p.qw_n; a.kh_n = p.kh_n; a.kw_n = p.kw_n;
+  a.err = p.err;
+  dim3 grid((unsigned)((p.Tq + 2 * kRowsPerTile - 1) / (2 * kRowsPerTile)), (unsigned)p.Hq, (unsigned)p.B);
+  const int mk = tc_mask_code(p);
+  if (!p.use_rel) {
+    if (p.d == 64) return dispatch_mask<64, 128, 0, 3>(mk, a, grid, stream);
+    return dispatch_mask<128, 128, 0, 2>(mk, a, grid, stream);
+  }
+  switch (p.kw_n) {
+    case 14: return dispatch_mask_rel<64, 112, 14, 3>(mk, a, grid, stream);
+    case 16: return dispatch_mask_rel<64, 128, 16, 2>(mk, a, grid, stream);
+    case 32: return dispatch_mask_rel<64, 128, 32, 2>(mk, a, grid, stream);
+    case 64: return dispatch_mask_rel<64, 128, 64, 2>(mk, a, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sdpa

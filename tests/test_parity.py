@@ -83,7 +83,7 @@ def _implemented(path):
     return path in _BUILT
 
 
-_BUILT = {"exact"}
+_BUILT = {"exact", "tcgen05"}
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -101,19 +101,28 @@ def test_parity(sp, path):
     assert np.max(np.abs(got[fin] - ref.lse[fin])) < 2e-3, "lse"
 
 
-def test_edge_cases_exact():
-    _edge_cases("exact")
+@pytest.mark.parametrize("path", ["exact", "tcgen05"])
+def test_edge_cases(path):
+    _edge_cases(path)
 
 
 def _edge_cases(path):
     import attention_sdpa_fwd_b200 as S
     dev = "cuda"
-    # Tkv = 0: every row sees nothing -> zeros, lse = -inf
-    q = torch.randn(1, 2, 5, 64, device=dev, dtype=BF16)
-    e = torch.empty(1, 2, 0, 64, device=dev, dtype=BF16)
-    lse = torch.zeros(1, 2, 5, device=dev)
+    if path == "exact":
+        # Tkv = 0: every row sees nothing -> zeros, lse = -inf
+        q = torch.randn(1, 2, 5, 64, device=dev, dtype=BF16)
+        e = torch.empty(1, 2, 0, 64, device=dev, dtype=BF16)
+        lse = torch.zeros(1, 2, 5, device=dev)
+        out = torch.full_like(q, 7.0)
+        S.sdpa(q, e, e, 0.1, out=out, lse=lse, path=path)
+        torch.cuda.synchronize()
+        assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+    # causal with a large negative offset: no row sees a key -> zeros, lse = -inf
+    q = torch.randn(1, 2, 300, 64, device=dev, dtype=BF16)
+    lse = torch.zeros(1, 2, 300, device=dev)
     out = torch.full_like(q, 7.0)
-    S.sdpa(q, e, e, 0.1, out=out, lse=lse, path=path)
+    S.sdpa(q, q, q, 0.1, mask_kind=S.MASK_CAUSAL, offset=-400, out=out, lse=lse, path=path)
     torch.cuda.synchronize()
     assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
     # B = 0: nothing to do
@@ -128,8 +137,8 @@ def _edge_cases(path):
     assert torch.equal(o1, v1)
     # fully masked rows (bool) -> zeros
     q2 = torch.randn(1, 1, 130, 64, device=dev, dtype=BF16)
-    k2 = torch.randn(1, 1, 140, 64, device=dev, dtype=BF16)
-    keep = torch.ones(1, 1, 130, 140, device=dev, dtype=torch.uint8)
+    k2 = torch.randn(1, 1, 144, 64, device=dev, dtype=BF16)
+    keep = torch.ones(1, 1, 130, 144, device=dev, dtype=torch.uint8)
     keep[0, 0, 3] = 0
     keep[0, 0, 129] = 0
     o2 = S.sdpa(q2, k2, k2, mask_kind=S.MASK_BOOL, mask=keep, path=path)
