@@ -17,9 +17,9 @@
 //   warp  8     TMA producer (Q once, then K_j / V_j per stage)
 //   warp  9     TMEM owner and MMA issuer (one elected thread)
 //   warps 10-11 idle
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D, 256+2D).
-// P (bf16) overwrites the first BN/2 columns of its S tile and is the A
-// operand of the P.V MMA straight from TMEM.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D, 256+2D);
+// P (bf16) is the A operand of the P.V MMA straight from TMEM: in its own
+// columns at head_dim 64, over the first BN/2 columns of its S tile at 128.
 //
 // Per KV tile j the MMA warp issues S_t = Q_t.K_j^T (SS, both K-major) and,
 // once softmax t has written P_t, O_t += P_t.V_j (TS, V MN-major).  The commit
@@ -48,6 +48,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;   // registers per thread the kernel is launched with
+constexpr int kRegsSoftmax = 224;  // after setmaxnreg, softmax warpgroups
+constexpr int kRegsOther = 56;     // after setmaxnreg, producer / MMA warpgroup
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch, "register split");
 constexpr int kRowsPerTile = 128;
 constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-pos path
 constexpr float kLog2e = 1.4426950408889634f;
@@ -68,6 +72,7 @@ struct TcArgs {
   float scale_log2;
   int qw_n, kh_n, kw_n;
   int rel_n;  // rows of the padded rel tables (multiple of 16, <= 128)
+  int mask_vec;  // mask rows allow 16-byte vector loads
   int* err;
 };
 
@@ -76,13 +81,13 @@ struct Layout {
   static constexpr int kPanels = D / 64;
   static constexpr int kQBytes = kPanels * kRowsPerTile * 128;  // one Q tile
   static constexpr int kKVBytes = kPanels * BN * 128;           // one K or V tile
-  static constexpr int kRelRows = KW > 0 ? kRelHMax + KW : 0;   // rel_h rows then rel_w rows, 256 floats each
+  static constexpr int kRelRows = KW > 0 ? kRelHMax + KW : 0;  // rel_h rows then rel_w rows, 256 floats each
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + 2 * kQBytes;
   static constexpr int oV = oK + NS * kKVBytes;
   static constexpr int oRel = oV + NS * kKVBytes;
   static constexpr int oBar = oRel + kRelRows * 256 * 4;
-  static constexpr int kBars = 3 * NS + 10;
+  static constexpr int kBars = 4 * NS + 14;
   static constexpr int kTotal = oBar + kBars * 8 + 16;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -92,6 +97,13 @@ struct Layout {
 template <int D, int BN, int KW, int MASK, int NS>
 __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constant__ TcArgs args) {
   using L = Layout<D, BN, KW, NS>;
+  // head_dim 64 leaves 128 TMEM columns free: P_A [384,448), P_B [448,512) get
+  // their own columns, so S_t(j+1) = Q_t.K_{j+1}^T can be issued as soon as
+  // softmax t has read S_t(j), before P_t(j) exists.  At head_dim 128, P_t
+  // overwrites S_t and the next Q.K^T waits for P_t.V.
+  constexpr bool kPSep = (D == 64);
+  constexpr bool kRwInSmem = KW >= 32;  // large key-grid width: rel_w re-read per tile
+  constexpr int kRwSwz = KW >= 64 ? 15 : 7;  // float4-index XOR swizzle of those rows (conflict-free)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::oQ;
@@ -101,14 +113,17 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::oBar);
   uint64_t* k_full = bars;               // [NS]  TMA -> MMA
   uint64_t* v_full = bars + NS;          // [NS]
-  uint64_t* kv_empty = bars + 2 * NS;    // [NS]  MMA commit -> TMA
-  uint64_t* q_full = bars + 3 * NS;      // Q tiles (and rel tables) landed
+  uint64_t* k_empty = bars + 2 * NS;     // [NS]  MMA commit after the last Q.K^T reading K -> TMA
+  uint64_t* v_empty = bars + 3 * NS;     // [NS]  MMA commit after the last P.V reading V -> TMA
+  uint64_t* q_full = bars + 4 * NS;      // Q tiles (and rel tables) landed
   uint64_t* s_full = q_full + 1;         // [2]   MMA commit -> softmax t
   uint64_t* p_full = q_full + 3;         // [2]   softmax t (128 arrivals) -> MMA
   uint64_t* o_done = q_full + 5;         // [2]   final MMA commit -> softmax t epilogue
   uint64_t* rel_mma = q_full + 7;        // rel projections in TMEM (MMA commit)
   uint64_t* rel_read = q_full + 8;       // projections read by all 256 softmax threads
   uint64_t* fin = q_full + 9;            // last commit before TMEM release
+  uint64_t* s_free = q_full + 10;        // [2]   softmax t read S_t (128 arrivals) -> MMA   (kPSep)
+  uint64_t* o_ready = q_full + 12;       // [2]   MMA commit after each O_t += P_t V         (kPSep)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + L::kBars);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
 
@@ -144,6 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     mbar_init(&p_full[0], kRowsPerTile);
     mbar_init(&p_full[1], kRowsPerTile);
     mbar_init(rel_read, 2 * kRowsPerTile);
+    mbar_init(&s_free[0], kRowsPerTile);
+    mbar_init(&s_free[1], kRowsPerTile);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -156,6 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   const uint32_t tbase = *tslot;
   volatile int* abort_v = abort_flag;
 
+  // Register split: the producer/MMA warpgroup gives registers to the two
+  // softmax warpgroups (3 x 128 x 168 at launch = 2 x 128 x 232 + 128 x 40).
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsOther));
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_tiles > 0) {
@@ -176,30 +197,44 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         tma_load_3d(sK + (NS - 1) * L::kKVBytes, &args.trh, q_full, 0, 0, 0);
         tma_load_3d(sV + (NS - 1) * L::kKVBytes, &args.trw, q_full, 0, 0, 0);
       }
+      // K runs one tile ahead of V: a K stage frees as soon as both Q.K^T
+      // products that read it are done, a V stage only after both P.V.
       bool ok = true;
-      int issued = 0;
-      for (int jj = 0; jj < n_tiles && ok; ++jj) {
-        const int s = jj % NS;
-        const int use = jj / NS;
-        if (use > 0) ok = mbar_wait(&kv_empty[s], (use - 1) & 1, abort_v, args.err);
+      int k_issued = 0, v_issued = 0;
+      auto load_k = [&](int jj) {
+        const int s = jj % NS, use = jj / NS;
+        if (use > 0) ok = mbar_wait(&k_empty[s], (use - 1) & 1, abort_v, args.err);
         if (ok && KW > 0 && jj == NS - 1) ok = mbar_wait(rel_mma, 0, abort_v, args.err);
-        if (!ok) break;
+        if (!ok) return;
         const int key0 = (j_begin + jj) * BN;
         mbar_expect_tx(&k_full[s], L::kKVBytes);
         for (int p = 0; p < L::kPanels; ++p)
           tma_load_3d(sK + s * L::kKVBytes + p * BN * 128, &args.tk, &k_full[s], p * 64, key0, zk);
+        k_issued = jj + 1;
+      };
+      auto load_v = [&](int jj) {
+        const int s = jj % NS, use = jj / NS;
+        if (use > 0) ok = mbar_wait(&v_empty[s], (use - 1) & 1, abort_v, args.err);
+        if (ok && KW > 0 && jj == NS - 1) ok = mbar_wait(rel_mma, 0, abort_v, args.err);
+        if (!ok) return;
+        const int key0 = (j_begin + jj) * BN;
         mbar_expect_tx(&v_full[s], L::kKVBytes);
         for (int p = 0; p < L::kPanels; ++p)
           tma_load_3d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, zk);
-        issued = jj + 1;
+        v_issued = jj + 1;
+      };
+      for (int jj = 0; jj < n_tiles && ok; ++jj) {
+        load_k(jj);
+        if (ok && jj > 0) load_v(jj - 1);
       }
+      if (ok) load_v(n_tiles - 1);
       if (!ok) {
         // abandoned: let the copies already in flight land before the CTA exits
         mbar_wait(q_full, 0, nullptr, args.err);
-        for (int jj = max(0, issued - NS); jj < issued; ++jj) {
+        for (int jj = max(0, k_issued - NS); jj < k_issued; ++jj)
           mbar_wait(&k_full[jj % NS], (jj / NS) & 1, nullptr, args.err);
+        for (int jj = max(0, v_issued - NS); jj < v_issued; ++jj)
           mbar_wait(&v_full[jj % NS], (jj / NS) & 1, nullptr, args.err);
-        }
       }
     }
   } else if (warp == 9) {
@@ -207,39 +242,43 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t id_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t id_pv = idesc_bf16_f32(128, D, false, true);
-      const uint32_t sq = smem_u32(sQ), sk = smem_u32(sK), sv = smem_u32(sV);
+      // Descriptors are built once; a byte offset inside shared memory is added
+      // to the start-address field (address >> 4, no carry out of 14 bits).
+      const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(sV), BN * 128, 1024);
       bool ok = mbar_wait(q_full, 0, abort_v, args.err);
       auto qk = [&](int t, int s) {
+        const uint64_t a0 = dq + (uint64_t)((t * L::kQBytes) >> 4);
+        const uint64_t b0 = dk + (uint64_t)((s * L::kKVBytes) >> 4);
+        const uint32_t d_tm = tbase + t * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;
-          const uint32_t a = sq + t * L::kQBytes + (kk >> 2) * (kRowsPerTile * 128) + koff;
-          const uint32_t bb = sk + s * L::kKVBytes + (kk >> 2) * (BN * 128) + koff;
-          mma_ss(tbase + t * 128, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id_qk, kk > 0);
+          const uint32_t ao = ((kk >> 2) * (kRowsPerTile * 128) + (kk & 3) * 32) >> 4;
+          const uint32_t bo = ((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4;
+          mma_ss(d_tm, a0 + ao, b0 + bo, id_qk, kk > 0);
         }
       };
       auto pv = [&](int t, int s, bool first) {
+        const uint64_t b0 = dv + (uint64_t)((s * L::kKVBytes) >> 4);
+        const uint32_t d_tm = tbase + 256 + t * D;
+        const uint32_t a_tm = kPSep ? tbase + 384 + t * 64 : tbase + t * 128;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t bb = sv + s * L::kKVBytes + kk * 16 * 128;
-          mma_ts(tbase + 256 + t * D, tbase + t * 128 + kk * 8, sdesc_sw128(bb, BN * 128, 1024), id_pv,
-                 (!first) || kk > 0);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d_tm, a_tm + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (!first) || kk > 0);
       };
       if (ok && KW > 0) {
         // rel projections: Ph_t -> cols [256t, 256t+rel_n), Pw_t -> [256t+128, 256t+128+rel_n)
         const uint32_t id_rel = idesc_bf16_f32(128, args.rel_n, false, false);
-        const uint32_t rh = sk + (NS - 1) * L::kKVBytes, rw = sv + (NS - 1) * L::kKVBytes;
+        const uint64_t drh = dk + (uint64_t)(((NS - 1) * L::kKVBytes) >> 4);
+        const uint64_t drw = sdesc_sw128(smem_u32(sV + (NS - 1) * L::kKVBytes), 16, 1024);
         tc_fence_after();
         for (int t = 0; t < 2; ++t)
           for (int w = 0; w < 2; ++w)
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t a = sq + t * L::kQBytes + kk * 32;
-              const uint32_t bb = (w == 0 ? rh : rw) + kk * 32;
-              mma_ss(tbase + t * 256 + w * 128, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id_rel,
-                     kk > 0);
-            }
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tbase + t * 256 + w * 128, dq + (uint64_t)((t * L::kQBytes + kk * 32) >> 4),
+                     (w == 0 ? drh : drw) + (uint64_t)((kk * 32) >> 4), id_rel, kk > 0);
         mma_commit(rel_mma);
         ok = mbar_wait(rel_read, 0, abort_v, args.err);
       }
@@ -251,40 +290,81 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         mma_commit(&s_full[0]);
         qk(1, 0);
         mma_commit(&s_full[1]);
+        mma_commit(&k_empty[0]);
       }
-      for (int jj = 0; jj < n_tiles && ok; ++jj) {
-        const int s = jj % NS;
-        ok = mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err);
-        if (!ok) break;
-        // tile A: O_A += P_A V_j, then S_A(j+1)
-        ok = mbar_wait(&p_full[0], jj & 1, abort_v, args.err);
-        if (!ok) break;
-        tc_fence_after();
-        pv(0, s, jj == 0);
-        const bool more = jj + 1 < n_tiles;
-        const int s1 = (jj + 1) % NS;
-        if (more) {
-          ok = mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err);
+      if constexpr (kPSep) {
+        // A and B alternate: S_A(j+1), O_A += P_A(j).V_j, S_B(j+1), O_B += P_B(j).V_j
+        for (int jj = 0; jj < n_tiles && ok; ++jj) {
+          const int s = jj % NS;
+          const bool more = jj + 1 < n_tiles;
+          const int s1 = (jj + 1) % NS;
+          if (more) {
+            ok = mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err);
+            if (ok) ok = mbar_wait(&s_free[0], jj & 1, abort_v, args.err);
+            if (!ok) break;
+            tc_fence_after();
+            qk(0, s1);
+            mma_commit(&s_full[0]);
+          }
+          ok = mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err);
+          if (ok) ok = mbar_wait(&p_full[0], jj & 1, abort_v, args.err);
           if (!ok) break;
           tc_fence_after();
-          qk(0, s1);
-          mma_commit(&s_full[0]);
+          pv(0, s, jj == 0);
+          mma_commit(&o_ready[0]);
+          if (more) {
+            ok = mbar_wait(&s_free[1], jj & 1, abort_v, args.err);
+            if (!ok) break;
+            tc_fence_after();
+            qk(1, s1);
+            mma_commit(&s_full[1]);
+            mma_commit(&k_empty[s1]);
+          }
+          ok = mbar_wait(&p_full[1], jj & 1, abort_v, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          pv(1, s, jj == 0);
+          mma_commit(&o_ready[1]);
+          mma_commit(&v_empty[s]);
         }
-        // tile B: O_B += P_B V_j, release stage j, then S_B(j+1)
-        ok = mbar_wait(&p_full[1], jj & 1, abort_v, args.err);
-        if (!ok) break;
-        tc_fence_after();
-        pv(1, s, jj == 0);
-        mma_commit(&kv_empty[s]);
-        if (more) {
-          qk(1, s1);
-          mma_commit(&s_full[1]);
+      } else {
+        for (int jj = 0; jj < n_tiles && ok; ++jj) {
+          const int s = jj % NS;
+          ok = mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err);
+          if (!ok) break;
+          // tile A: O_A += P_A V_j, then S_A(j+1)
+          ok = mbar_wait(&p_full[0], jj & 1, abort_v, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          pv(0, s, jj == 0);
+          const bool more = jj + 1 < n_tiles;
+          const int s1 = (jj + 1) % NS;
+          if (more) {
+            ok = mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err);
+            if (!ok) break;
+            tc_fence_after();
+            qk(0, s1);
+            mma_commit(&s_full[0]);
+          }
+          // tile B: O_B += P_B V_j, release V_j, then S_B(j+1) and release K_{j+1}
+          ok = mbar_wait(&p_full[1], jj & 1, abort_v, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          pv(1, s, jj == 0);
+          mma_commit(&v_empty[s]);
+          if (more) {
+            qk(1, s1);
+            mma_commit(&s_full[1]);
+            mma_commit(&k_empty[s1]);
+          }
         }
       }
       mma_commit(&o_done[0]);
       mma_commit(&o_done[1]);
     }
-  } else if (warp < 8) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax of tile t
     const int t = warp >> 2;
     const int lr = (warp & 3) * 32 + lane;   // row within the tile = TMEM lane
@@ -293,9 +373,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_addr = tbase + lane_off + t * 128;
     const uint32_t o_addr = tbase + lane_off + 256 + t * D;
+    const uint32_t p_addr = kPSep ? tbase + lane_off + 384 + t * 64 : s_addr;
     bool ok = true;
-    float* relh_s = sRel;                  // [kRelHMax][256]
-    float* relw_s = sRel + kRelHMax * 256;  // [KW][256]
+    float* relh_s = sRel;                   // [kRelHMax][256]
+    float* relw_s = sRel + kRelHMax * 256;  // [KW][256], or [256][KW] (swizzled) when read as float4 per tile
 
     if constexpr (KW > 0) if (n_tiles > 0) {
       // scatter this row's rel_h / rel_w (log2 e prescaled) into shared memory
@@ -318,7 +399,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int k = base_idx - (c0 + i);  // key-grid coordinate reached through table row c0+i
-                if (k >= 0 && k < nk) dst[k * 256 + row] = __uint_as_float(r[i]) * kLog2e;
+                if (k >= 0 && k < nk) {
+                  // rel_w of a large grid: row-major per query row, float4 groups XOR-swizzled by row
+                  const int off = (w == 1 && kRwInSmem) ? row * KW + (((k >> 2) ^ (row & kRwSwz)) << 2) + (k & 3)
+                                                        : k * 256 + row;
+                  dst[off] = __uint_as_float(r[i]) * kLog2e;
+                }
               }
             }
           }
@@ -337,95 +423,151 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     const bool row_valid = qi < args.Tq;
     const long long mrow = (long long)b * args.msb + (long long)h * args.msh + qi * args.msq;
 
+    // rel_w of this row: in registers for the whole loop when small, else
+    // re-read per tile as float4 from this row's shared-memory slice (log2 units)
+    float rw[(KW > 0 && !kRwInSmem) ? KW : 2];
+    if constexpr (KW > 0 && !kRwInSmem) {
+#pragma unroll
+      for (int c = 0; c < KW; ++c) rw[c] = relw_s[c * 256 + row];
+    }
+    const float4* rw4 = reinterpret_cast<const float4*>(relw_s + row * (KW > 0 ? KW : 1));
+    constexpr int NG = KW > 0 ? BN / KW : 1;  // key-grid rows per key tile (1 without rel-pos)
+    constexpr int GW = BN / NG;                // keys per group
+    static_assert(GW % 2 == 0, "groups hold whole pairs");
+    const uint64_t sl2 = f2(args.scale_log2, args.scale_log2);
+
     float m_run = -INFINITY, l_run = 0.f;
     for (int jj = 0; jj < n_tiles && ok; ++jj) {
       const int j0 = (j_begin + jj) * BN;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], jj & 1, abort_v, args.err));
       if (!ok) break;
       tc_fence_after();
-      float x[BN];
+      uint32_t sr[BN];
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) {
-        if (c0 + 32 <= BN) {
-          uint32_t r[32];
-          tmem_ld32(s_addr + c0, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[c0 + i] = __uint_as_float(r[i]);
-        } else {
-          uint32_t r[16];
-          tmem_ld16(s_addr + c0, r);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) x[c0 + i] = __uint_as_float(r[i]);
-        }
+        if (c0 + 32 <= BN)
+          tmem_ld32p(s_addr + c0, sr + c0);
+        else
+          tmem_ld16p(s_addr + c0, sr + c0);
       }
       tmem_wait_ld();
+      if constexpr (kPSep) {
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);
+      }
 
-      // scale (and rel-pos bias), in log2 units
+      // x = s*scale (+ rel_w) in log2 units, two columns per instruction; rel_h
+      // is constant over a key-grid row, so it is kept per group (goff) and
+      // folded into the max and the exponent.
+      uint64_t x2[BN / 2];
+      float goff[NG];
       if constexpr (KW > 0) {
         const int kh0 = j0 / KW;
 #pragma unroll
-        for (int g = 0; g < BN / KW; ++g) {
+        for (int g = 0; g < NG; ++g) {
           const int khi = kh0 + g;
-          const float rh = khi < args.kh_n ? relh_s[khi * 256 + row] : 0.f;
+          goff[g] = khi < args.kh_n ? relh_s[khi * 256 + row] : 0.f;
+        }
+        if constexpr (kRwInSmem) {
 #pragma unroll
-          for (int c = 0; c < KW; ++c)
-            x[g * KW + c] = fmaf(x[g * KW + c], args.scale_log2, relw_s[c * 256 + row] + rh);
+          for (int c = 0; c < KW; c += 4) {
+            const float4 w4 = rw4[(c / 4) ^ (row & kRwSwz)];
+            const uint64_t wa = f2(w4.x, w4.y), wb = f2(w4.z, w4.w);
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+              const int e = g * KW + c;
+              x2[e / 2] = f2_fma(f2u(sr[e], sr[e + 1]), sl2, wa);
+              x2[e / 2 + 1] = f2_fma(f2u(sr[e + 2], sr[e + 3]), sl2, wb);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int c = 0; c < KW; c += 2) {
+              const int e = g * KW + c;
+              x2[e / 2] = f2_fma(f2u(sr[e], sr[e + 1]), sl2, f2(rw[c], rw[c + 1]));
+            }
         }
       } else {
+        goff[0] = 0.f;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) x[c] *= args.scale_log2;
+        for (int i = 0; i < BN / 2; ++i) x2[i] = f2_mul(f2u(sr[2 * i], sr[2 * i + 1]), sl2);
       }
+
+      // masks (scalar, only on tiles that need them)
+      auto set_ninf = [&](int c) {
+        float lo, hi;
+        f2_split(x2[c / 2], lo, hi);
+        if (c & 1) hi = -INFINITY; else lo = -INFINITY;
+        x2[c / 2] = f2(lo, hi);
+      };
       if constexpr (MASK == TC_RANGE) {
         if (!(j0 >= lo_i && j0 + BN <= hi_i)) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
-            if (j0 + c < lo_i || j0 + c >= hi_i) x[c] = -INFINITY;
+            if (j0 + c < lo_i || j0 + c >= hi_i) set_ninf(c);
         }
       } else if constexpr (MASK == TC_FLOAT) {
         if (row_valid) {
-        const __nv_bfloat16* mp = static_cast<const __nv_bfloat16*>(args.mask) + mrow + j0;
-        if (j0 + BN <= args.Tkv) {
+          const __nv_bfloat16* mp = static_cast<const __nv_bfloat16*>(args.mask) + mrow + j0;
+          const uint64_t l2e = f2(kLog2e, kLog2e);
+          if (j0 + BN <= args.Tkv && args.mask_vec) {
 #pragma unroll
-          for (int c = 0; c < BN; c += 8) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(mp + c));
-            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+            for (int c = 0; c < BN; c += 8) {
+              const uint4 raw = __ldg(reinterpret_cast<const uint4*>(mp + c));
+              const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) x[c + u] = fmaf(__bfloat162float(e[u]), kLog2e, x[c + u]);
+              for (int u = 0; u < 4; ++u)  // bf16 pair -> fp32 pair by moving each half to the top 16 bits
+                x2[c / 2 + u] = f2_fma(f2u(wv[u] << 16, wv[u] & 0xFFFF0000u), l2e, x2[c / 2 + u]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN; c += 2) {
+              const float m0 = j0 + c < args.Tkv ? __bfloat162float(mp[c]) : 0.f;
+              const float m1 = j0 + c + 1 < args.Tkv ? __bfloat162float(mp[c + 1]) : 0.f;
+              x2[c / 2] = f2_fma(f2(m0, m1), l2e, x2[c / 2]);
+            }
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (j0 + c < args.Tkv) x[c] = fmaf(__bfloat162float(mp[c]), kLog2e, x[c]);
-        }
         }
       } else if constexpr (MASK == TC_BOOL) {
         if (row_valid) {
-        const uint8_t* mp = static_cast<const uint8_t*>(args.mask) + mrow + j0;
-        if (j0 + BN <= args.Tkv) {
+          const uint8_t* mp = static_cast<const uint8_t*>(args.mask) + mrow + j0;
+          if (j0 + BN <= args.Tkv && args.mask_vec) {
 #pragma unroll
-          for (int c = 0; c < BN; c += 16) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(mp + c));
-            const uint8_t* e = reinterpret_cast<const uint8_t*>(&raw);
+            for (int c = 0; c < BN; c += 16) {
+              const uint4 raw = __ldg(reinterpret_cast<const uint4*>(mp + c));
+              const uint8_t* e = reinterpret_cast<const uint8_t*>(&raw);
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              if (e[u] == 0) x[c + u] = -INFINITY;
+              for (int u = 0; u < 16; ++u)
+                if (e[u] == 0) set_ninf(c + u);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              if (j0 + c < args.Tkv && mp[c] == 0) set_ninf(c);
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (j0 + c < args.Tkv && mp[c] == 0) x[c] = -INFINITY;
-        }
         }
       }
       if (j0 + BN > args.Tkv) {
 #pragma unroll
         for (int c = 0; c < BN; ++c)
-          if (j0 + c >= args.Tkv) x[c] = -INFINITY;
+          if (j0 + c >= args.Tkv) set_ninf(c);
       }
 
+      // row max: three-input max over pairs, four independent chains per group
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      for (int g = 0; g < NG; ++g) {
+        float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < GW / 2; ++i) {
+          float lo, hi;
+          f2_split(x2[g * GW / 2 + i], lo, hi);
+          a[i & 3] = max3(a[i & 3], lo, hi);
+        }
+        mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) + goff[g]);
+      }
       const float m_new = fmaxf(m_run, mx);
       const bool need = m_new > m_run + kRescaleThreshold;  // false while both are -inf
       float alpha = 1.f;
@@ -433,6 +575,14 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         alpha = ex2_approx(m_run - m_new);  // 0 when m_run == -inf
         l_run *= alpha;
         m_run = m_new;
+      }
+      if constexpr (kPSep) {
+        // O_t += P_t(j-1).V_{j-1} must be complete before O_t is rescaled or P_t is overwritten
+        if (jj > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (jj - 1) & 1, abort_v, args.err));
+          if (!ok) break;
+          tc_fence_after();
+        }
       }
       if (jj > 0 && __any_sync(0xffffffffu, need)) {
         // O_t row *= alpha (warp-collective; alpha is 1 where the max did not move)
@@ -447,23 +597,30 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         }
       }
 
+      // p = 2^(x + goff - m), packed to bf16 pairs and written to P in TMEM
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      float rowsum = 0.f;
-      uint32_t pk[BN / 2];
+      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2_approx(x[c] - m_use);
-        const float p1 = ex2_approx(x[c + 1] - m_use);
-        rowsum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
-      }
-      l_run += rowsum;
-#pragma unroll
-      for (int c0 = 0; c0 < BN / 2; c0 += 8) {
+      for (int c0 = 0; c0 < BN; c0 += 16) {
         uint32_t r8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) r8[i] = pk[c0 + i];
-        tmem_st8(s_addr + c0, r8);
+        for (int i = 0; i < 8; ++i) {
+          const int c = c0 + 2 * i;
+          const float nmo = goff[c / GW] - m_use;
+          float lo, hi;
+          f2_split(f2_add(x2[c / 2], f2(nmo, nmo)), lo, hi);
+          const float p0 = ex2_approx(lo);
+          const float p1 = ex2_approx(hi);
+          sum2[i & 1] = f2_add(sum2[i & 1], f2(p0, p1));
+          r8[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st8(p_addr + c0 / 2, r8);
+      }
+      {
+        float a0, a1, b0, b1;
+        f2_split(sum2[0], a0, a1);
+        f2_split(sum2[1], b0, b1);
+        l_run += (a0 + a1) + (b0 + b1);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -480,7 +637,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         if (args.lse) args.lse[zq * args.Tq + qi] = -INFINITY;
       }
     } else {
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, abort_v, args.err));
+      if (ok) {
+        if constexpr (kPSep)
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (n_tiles - 1) & 1, abort_v, args.err));
+        else
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, abort_v, args.err));
+      }
       tc_fence_after();
       if (ok) {
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -531,6 +693,11 @@ cudaError_t launch_one(const TcArgs& a, dim3 grid, cudaStream_t stream) {
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    // setmaxnreg.inc waits for registers the CTA was launched with: refuse to
+    // launch unless the split adds up against the compiled register count.
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, kern);
+    if (attr_err == cudaSuccess && fa.numRegs != kRegsLaunch) attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, kThreads, L::kAlloc, stream>>>(a);
@@ -591,12 +758,6 @@ int tc_check(const Params& p, sdpa_dtype_t dtype) {
     if (p.mask_kind == SDPA_MASK_ADD_FLOAT || p.mask_kind == SDPA_MASK_BOOL) return SDPA_ERR_UNSUPPORTED;
     if (!al16(p.rel_h) || !al16(p.rel_w)) return SDPA_ERR_MISALIGNED;
   }
-  if (p.mask_kind == SDPA_MASK_ADD_FLOAT) {
-    if (!al16(p.mask) || (p.msb % 8) || (p.msh % 8) || (p.msq % 8)) return SDPA_ERR_MISALIGNED;
-  }
-  if (p.mask_kind == SDPA_MASK_BOOL) {
-    if (!al16(p.mask) || (p.msb % 16) || (p.msh % 16) || (p.msq % 16)) return SDPA_ERR_MISALIGNED;
-  }
   return SDPA_OK;
 }
 
@@ -624,6 +785,10 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   a.offset = p.offset; a.window = p.window;
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.Tq = p.Tq; a.Tkv = p.Tkv; a.group = p.group;
   a.mask_kind = p.mask_kind;
+  if (p.mask_kind == SDPA_MASK_ADD_FLOAT)
+    a.mask_vec = al16(p.mask) && !(p.msb % 8) && !(p.msh % 8) && !(p.msq % 8);
+  if (p.mask_kind == SDPA_MASK_BOOL)
+    a.mask_vec = al16(p.mask) && !(p.msb % 16) && !(p.msh % 16) && !(p.msq % 16);
   a.scale_log2 = p.scale * kLog2e;
   a.qw_n = p.qw_n; a.kh_n = p.kh_n; a.kw_n = p.kw_n;
   a.err = p.err;

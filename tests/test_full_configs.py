@@ -31,4 +31,4 @@ def test_full_size(sp):
                                                           sp.window + 1) if sp.window else ())
         ref = oracle_ref(wl, rows=rows)
         got = out[:, :, rows].double().numpy()
-    assert_gates(got, ref.out, sp.dtype, sp.name)
+    assert_gates(got, ref.out, sp.dtype, sp.name, strong=sp.name.endswith("_strong"))

@@ -57,6 +57,22 @@ CASES = [
     S_("bool_bf16_d128_bcast", BF16, 1, 4, 4, 130, 128, 128, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.9,
        mask_heads=1, seed=25),
     S_("mqa_bf16_d128", BF16, 2, 8, 1, 200, 256, 128, seed=26),
+    # rel-pos shapes the tensor-core path specialises (key-grid width 14/16/32/64)
+    S_("relpos_bf16_d64_12x16", BF16, 2, 3, 3, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5, seed=27),
+    S_("relpos_bf16_d64_8x32", BF16, 1, 4, 2, 256, 256, 64, q_hw=(8, 32), k_hw=(8, 32), rel_std=0.5, seed=28),
+    S_("relpos_bf16_d64_20x14", BF16, 3, 2, 2, 280, 280, 64, q_hw=(20, 14), k_hw=(20, 14), rel_std=0.5, seed=29),
+    S_("relpos_bf16_d64_9x64", BF16, 1, 2, 2, 576, 576, 64, q_hw=(9, 64), k_hw=(9, 64), rel_std=0.5, seed=30),
+    S_("relpos_bf16_d64_14x14_strong", BF16, 7, 3, 3, 196, 196, 64, q_hw=(14, 14), k_hw=(14, 14), rel_std=1.0,
+       seed=31),
+    # rel-pos combined with a causal / sliding mask
+    S_("relpos_causal_bf16_d64_12x16", BF16, 1, 2, 2, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5,
+       mask_kind=W.MASK_CAUSAL, seed=32),
+    S_("relpos_sliding_bf16_d64_20x14", BF16, 1, 2, 2, 280, 280, 64, q_hw=(20, 14), k_hw=(20, 14), rel_std=0.5,
+       mask_kind=W.MASK_SLIDING, window=60, offset=3, seed=33),
+    S_("float_bf16_d64_aligned", BF16, 2, 2, 1, 300, 296, 64, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=2, seed=34),
+    S_("bool_bf16_d128_aligned", BF16, 1, 2, 2, 260, 272, 128, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.5,
+       mask_heads=1, seed=35),
 ]
 CASE_IDS = [c.name for c in CASES]
 
@@ -70,7 +86,15 @@ def applicable(path: str, sp: W.Spec) -> bool:
     if sp.dtype != BF16:
         return False
     if path == "tcgen05":
-        return sp.d in (64, 128)
+        if sp.d not in (64, 128):
+            return False
+        if sp.rel:
+            kh, kw = sp.k_hw
+            bn = 112 if kw == 14 else 128
+            return (sp.d == 64 and kw in (14, 16, 32, 64) and kh <= 64
+                    and ((2 * max(kh, kw) - 1) + 15) // 16 * 16 <= bn
+                    and sp.mask_kind in (W.MASK_NONE, W.MASK_CAUSAL, W.MASK_SLIDING))
+        return True
     if path == "small_d":
         return sp.d == 16
     if path == "split_kv":
@@ -94,7 +118,7 @@ def test_parity(sp, path):
     wl = W.make(sp)
     out, lse = gpu_run(wl, path=path, want_lse=True)
     ref = oracle_ref(wl)
-    assert_gates(out.double().numpy(), ref.out, sp.dtype, f"{sp.name}/{path}")
+    assert_gates(out.double().numpy(), ref.out, sp.dtype, f"{sp.name}/{path}", strong=sp.name.endswith("_strong"))
     fin = np.isfinite(ref.lse)
     got = lse.double().numpy()
     assert np.array_equal(np.isfinite(got), fin), "lse -inf pattern"
