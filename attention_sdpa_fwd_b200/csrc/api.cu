@@ -34,6 +34,21 @@ int* error_word_ptr() {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Scratch for split key ranges, one per device, grown on demand and never
+// shrunk: a counter area that is zero between launches (every kernel that
+// takes tickets from it puts them back to zero) and a separate data area for
+// partial results.  `dirty` is set when a kernel may have left counters
+// non-zero (a device-side wait gave up); the next user clears them first.
+struct Workspace {
+  void* cnt = nullptr;
+  size_t cnt_cap = 0;
+  void* data = nullptr;
+  size_t data_cap = 0;
+  bool dirty = false;
+};
+Workspace g_ws[kMaxDevices];
+std::mutex g_ws_mu;
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
   uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -123,7 +138,14 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
 }
 
 int choose_path(const Problem& pr) {
-  if (tc_check(pr.p, pr.dtype) == SDPA_OK) return SDPA_PATH_TCGEN05;
+  const Params& p = pr.p;
+  if (p.Tkv == 0) return SDPA_PATH_EXACT;
+  if (tc_check(p, pr.dtype) == SDPA_OK) return SDPA_PATH_TCGEN05;
+  if (small_d_check(p, pr.dtype) == SDPA_OK) {
+    // few query rows against a long key axis: split the keys over the SMs
+    if (p.Tq <= 64 && p.Tkv >= 1024) return SDPA_PATH_SPLIT_KV;
+    return SDPA_PATH_SMALL_D;
+  }
   return SDPA_PATH_EXACT;
 }
 
@@ -142,14 +164,80 @@ int run(const Problem& pr, int path, cudaStream_t stream) {
       e = launch_tc(p, stream);
       break;
     }
-    case SDPA_PATH_SMALL_D:
-    case SDPA_PATH_SPLIT_KV: return SDPA_ERR_UNSUPPORTED;
+    case SDPA_PATH_SMALL_D: {
+      const int rc = small_d_check(p, pr.dtype);
+      if (rc != SDPA_OK) return rc;
+      e = launch_small_d(p, stream);
+      break;
+    }
+    case SDPA_PATH_SPLIT_KV: {
+      const int rc = split_kv_check(p, pr.dtype);
+      if (rc != SDPA_OK) return rc;
+      e = launch_split_kv(p, stream);
+      break;
+    }
     default: return SDPA_ERR_INVALID_ARG;
   }
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }
 
 }  // namespace
+
+int workspace_get(size_t cnt_bytes, size_t data_bytes, void** cnt, void** data, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SDPA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  Workspace& w = g_ws[dev];
+  auto round_mb = [](size_t x) { return (x + (1u << 20) - 1) & ~size_t((1u << 20) - 1); };
+  if (w.cnt_cap < cnt_bytes || w.data_cap < data_bytes) {
+    // earlier launches may still use the old buffers
+    if ((w.cnt || w.data) && cudaDeviceSynchronize() != cudaSuccess) return SDPA_ERR_CUDA;
+  }
+  if (w.cnt_cap < cnt_bytes) {
+    if (w.cnt) cudaFree(w.cnt);
+    w.cnt = nullptr;
+    w.cnt_cap = 0;
+    const size_t cap = round_mb(cnt_bytes);
+    if (cudaMalloc(&w.cnt, cap) != cudaSuccess) return SDPA_ERR_CUDA;
+    if (cudaMemset(w.cnt, 0, cap) != cudaSuccess) return SDPA_ERR_CUDA;
+    w.cnt_cap = cap;
+  }
+  if (w.data_cap < data_bytes) {
+    if (w.data) cudaFree(w.data);
+    w.data = nullptr;
+    w.data_cap = 0;
+    const size_t cap = round_mb(data_bytes);
+    if (cudaMalloc(&w.data, cap) != cudaSuccess) return SDPA_ERR_CUDA;
+    w.data_cap = cap;
+  }
+  if (w.dirty) {
+    if (cudaMemsetAsync(w.cnt, 0, w.cnt_cap, stream) != cudaSuccess) return SDPA_ERR_CUDA;
+    w.dirty = false;
+  }
+  *cnt = w.cnt;
+  *data = w.data;
+  return SDPA_OK;
+}
+
+int num_sms() {
+  static int cached[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+void mark_workspace_dirty() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  g_ws[dev].dirty = true;
+}
+
 }  // namespace sdpa
 
 using namespace sdpa;
@@ -280,6 +368,7 @@ extern "C" int sdpa_last_device_error(cudaStream_t stream) {
   if (host != 0) {
     const int zero = 0;
     if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SDPA_ERR_CUDA;
+    mark_workspace_dirty();  // an abandoned split may have left its counters behind
     return SDPA_ERR_TIMEOUT;
   }
   return SDPA_OK;

@@ -61,6 +61,20 @@ __host__ __device__ __forceinline__ void key_range(const Params& p, long long i,
 // Launchers (one per kernel family); each returns a cudaError_t of the launch.
 cudaError_t launch_exact(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
 int tc_check(const Params& p, sdpa_dtype_t dtype);  // SDPA_OK or why the tensor-core kernel cannot run
+// Library-owned scratch of the current device: a counter area of at least
+// `cnt_bytes` that is zero when the next kernel on `stream` starts (kernels
+// taking tickets from it leave it zero again) and a data area of at least
+// `data_bytes`.  Returns SDPA_OK or SDPA_ERR_CUDA.
+int workspace_get(size_t cnt_bytes, size_t data_bytes, void** cnt, void** data, cudaStream_t stream);
+int small_d_check(const Params& p, sdpa_dtype_t dtype);
+cudaError_t launch_small_d(const Params& p, cudaStream_t stream);
+int split_kv_check(const Params& p, sdpa_dtype_t dtype);
+cudaError_t launch_split_kv(const Params& p, cudaStream_t stream);
+// scratch the split-KV kernel needs for this problem (tickets that must be
+// zero at launch, and partial results) and the launch on given scratch
+void split_kv_workspace_bytes(const Params& p, size_t* cnt_bytes, size_t* data_bytes);
+cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream_t stream);
+int num_sms();
 cudaError_t launch_tc(const Params& p, cudaStream_t stream);
 
 }  // namespace sdpa

@@ -73,6 +73,10 @@ struct TcArgs {
   int qw_n, kh_n, kw_n;
   int rel_n;  // rows of the padded rel tables (multiple of 16, <= 128)
   int mask_vec;  // mask rows allow 16-byte vector loads
+  int n_split;   // CTAs sharing one 256-row query block (key range split); 1 = no split
+  float* ws_o;   // [blocks][n_split][256][D] unnormalised partial outputs   (n_split > 1)
+  float2* ws_ml; // [blocks][n_split][256] (running max in log2 units, sum)   (n_split > 1)
+  int* ws_cnt;   // [blocks] arrival counters, zero between launches         (n_split > 1)
   int* err;
 };
 
@@ -88,11 +92,15 @@ struct Layout {
   static constexpr int oRel = oV + NS * kKVBytes;
   static constexpr int oBar = oRel + kRelRows * 256 * 4;
   static constexpr int kBars = 4 * NS + 14;
-  static constexpr int kTotal = oBar + kBars * 8 + 16;
+  static constexpr int kTotal = oBar + kBars * 8 + 32;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
   static_assert(KW == 0 || (BN % (KW > 0 ? KW : 1) == 0), "key tile must hold whole key-grid rows");
 };
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 template <int D, int BN, int KW, int MASK, int NS>
 __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constant__ TcArgs args) {
@@ -130,14 +138,16 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int qblk = blockIdx.x;
+  const int nsplit = args.n_split;
+  const int qblk = blockIdx.x / nsplit;
+  const int sidx = blockIdx.x - qblk * nsplit;  // which part of the key range this CTA takes
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int hk = h / args.group;
   const int q0 = qblk * 2 * kRowsPerTile;
 
-  // Key-tile range of this CTA (causal / sliding skip whole tiles).
-  int j_begin = 0, j_end = (args.Tkv + BN - 1) / BN;
+  // Key-tile range of the query block (causal / sliding skip whole tiles) ...
+  int jb = 0, je = (args.Tkv + BN - 1) / BN;
   if (MASK == TC_RANGE) {
     const long long first = q0;
     const long long last = (long long)min(q0 + 2 * kRowsPerTile, args.Tq) - 1;
@@ -145,12 +155,15 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     if (last + args.offset + 1 < hi) hi = last + args.offset + 1;
     if (args.mask_kind == SDPA_MASK_SLIDING) lo = max(0LL, first + args.offset - args.window + 1);
     if (hi <= lo) {
-      j_begin = j_end = 0;
+      jb = je = 0;
     } else {
-      j_begin = (int)(lo / BN);
-      j_end = (int)((hi + BN - 1) / BN);
+      jb = (int)(lo / BN);
+      je = (int)((hi + BN - 1) / BN);
     }
   }
+  // ... and this CTA's share of it
+  const int j_begin = jb + (int)((long long)(je - jb) * sidx / nsplit);
+  const int j_end = jb + (int)((long long)(je - jb) * (sidx + 1) / nsplit);
   const int n_tiles = j_end - j_begin;
 
   if (tid == 0) {
@@ -399,16 +412,25 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int k = base_idx - (c0 + i);  // key-grid coordinate reached through table row c0+i
-                if (k >= 0 && k < nk) {
-                  // rel_w of a large grid: row-major per query row, float4 groups XOR-swizzled by row
-                  const int off = (w == 1 && kRwInSmem) ? row * KW + (((k >> 2) ^ (row & kRwSwz)) << 2) + (k & 3)
-                                                        : k * 256 + row;
-                  dst[off] = __uint_as_float(r[i]) * kLog2e;
-                }
+                // [k][256] layout: consecutive rows hit consecutive banks whatever k is
+                if (k >= 0 && k < nk) dst[k * 256 + row] = __uint_as_float(r[i]) * kLog2e;
               }
             }
           }
         }
+      }
+      if constexpr (kRwInSmem) {
+        // Large key-grid width: the loop re-reads rel_w per tile as float4, so
+        // move this row's values into a row-major slice with float4 groups
+        // XOR-swizzled by row (conflict-free 128-bit reads), via registers.
+        float v[KW];
+#pragma unroll
+        for (int k = 0; k < KW; ++k) v[k] = relw_s[k * 256 + row];
+        named_bar_sync(1, 2 * kRowsPerTile);
+#pragma unroll
+        for (int k = 0; k < KW; k += 4)
+          *reinterpret_cast<float4*>(relw_s + row * KW + (((k >> 2) ^ (row & kRwSwz)) << 2)) =
+              make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
       }
       tc_fence_before();
       mbar_arrive(rel_read);
@@ -630,21 +652,21 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     // epilogue: O / l -> bf16, rows past Tq are not stored
     const long long zq = (long long)b * args.Hq + h;
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (zq * args.Tq + qi) * D;
-    if (n_tiles == 0) {
-      if (row_valid) {
-#pragma unroll
-        for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-        if (args.lse) args.lse[zq * args.Tq + qi] = -INFINITY;
-      }
-    } else {
-      if (ok) {
-        if constexpr (kPSep)
-          ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (n_tiles - 1) & 1, abort_v, args.err));
-        else
-          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, abort_v, args.err));
-      }
+    if (n_tiles > 0 && ok) {
+      if constexpr (kPSep)
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (n_tiles - 1) & 1, abort_v, args.err));
+      else
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, abort_v, args.err));
       tc_fence_after();
-      if (ok) {
+    }
+    if (nsplit == 1) {
+      if (n_tiles == 0) {
+        if (row_valid) {
+#pragma unroll
+          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+          if (args.lse) args.lse[zq * args.Tq + qi] = -INFINITY;
+        }
+      } else if (ok) {
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -665,6 +687,75 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         }
         if (row_valid && args.lse)
           args.lse[zq * args.Tq + qi] = l_run > 0.f ? m_run * kLn2 + logf(l_run) : -INFINITY;
+      }
+    } else {
+      // Split key range: publish this part (O unnormalised, running max m in
+      // log2 units, sum l); the last CTA of the block to arrive combines the
+      // parts, O = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k with M = max_k m_k.
+      const long long blk = zq * (gridDim.x / nsplit) + qblk;
+      float* wso = args.ws_o + ((blk * nsplit + sidx) * 256 + row) * D;
+      const bool have = n_tiles > 0 && ok && l_run > 0.f;
+      if (n_tiles > 0 && ok) {  // warp-uniform: the TMEM load is warp-collective
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c0, r);
+          tmem_wait_ld();
+          if (have) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              __stcg(reinterpret_cast<float4*>(wso + c0 + c),
+                     make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
+                                 __uint_as_float(r[c + 3])));
+          }
+        }
+      }
+      __stcg(args.ws_ml + (blk * nsplit + sidx) * 256 + row, make_float2(have ? m_run : -INFINITY, have ? l_run : 0.f));
+      __threadfence();
+      named_bar_sync(1, 2 * kRowsPerTile);
+      if (tid == 0) *reinterpret_cast<volatile int*>(abort_flag + 1) = atomicAdd(args.ws_cnt + blk, 1) == nsplit - 1;
+      named_bar_sync(1, 2 * kRowsPerTile);
+      if (*reinterpret_cast<volatile int*>(abort_flag + 1)) {
+        __threadfence();
+        float M = -INFINITY;
+        for (int k = 0; k < nsplit; ++k) {
+          const float2 ml = __ldcg(args.ws_ml + (blk * nsplit + k) * 256 + row);
+          if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        }
+        float acc[D];
+#pragma unroll
+        for (int c = 0; c < D; ++c) acc[c] = 0.f;
+        float den = 0.f;
+        for (int k = 0; k < nsplit; ++k) {
+          const float2 ml = __ldcg(args.ws_ml + (blk * nsplit + k) * 256 + row);
+          if (ml.y > 0.f) {
+            const float w = ex2_approx(ml.x - M);
+            den = fmaf(w, ml.y, den);
+            const float* src = args.ws_o + ((blk * nsplit + k) * 256 + row) * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 4) {
+              const float4 o4 = __ldcg(reinterpret_cast<const float4*>(src + c));
+              acc[c] = fmaf(w, o4.x, acc[c]);
+              acc[c + 1] = fmaf(w, o4.y, acc[c + 1]);
+              acc[c + 2] = fmaf(w, o4.z, acc[c + 2]);
+              acc[c + 3] = fmaf(w, o4.w, acc[c + 3]);
+            }
+          }
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        if (row_valid) {
+#pragma unroll
+          for (int c = 0; c < D; c += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(acc[c + 0] * inv, acc[c + 1] * inv);
+            v.y = pack_bf16x2(acc[c + 2] * inv, acc[c + 3] * inv);
+            v.z = pack_bf16x2(acc[c + 4] * inv, acc[c + 5] * inv);
+            v.w = pack_bf16x2(acc[c + 6] * inv, acc[c + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + c) = v;
+          }
+          if (args.lse) args.lse[zq * args.Tq + qi] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
+        }
+        if (tid == 0) args.ws_cnt[blk] = 0;  // ready for the next launch
       }
     }
   }
@@ -792,8 +883,36 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   a.scale_log2 = p.scale * kLog2e;
   a.qw_n = p.qw_n; a.kh_n = p.kh_n; a.kw_n = p.kw_n;
   a.err = p.err;
-  dim3 grid((unsigned)((p.Tq + 2 * kRowsPerTile - 1) / (2 * kRowsPerTile)), (unsigned)p.Hq, (unsigned)p.B);
+  const int nqblk = (p.Tq + 2 * kRowsPerTile - 1) / (2 * kRowsPerTile);
   const int mk = tc_mask_code(p);
+  // Fewer than two waves of query blocks: split each block's key range over
+  // several CTAs so the waves fill the SMs (parts merged in-kernel).
+  a.n_split = 1;
+  const long long nblk = (long long)nqblk * p.Hq * p.B;
+  const int nsm = num_sms();
+  const int nt = (p.Tkv + BN - 1) / BN;
+  if (mk != TC_RANGE && nblk < 2LL * nsm && nt >= 2) {
+    double best = 1e30;
+    for (int sp = 1; sp <= 8 && sp <= nt; ++sp) {
+      const double waves = (double)((nblk * sp + nsm - 1) / nsm);
+      const double cost = waves * ((nt + sp - 1) / sp + 1.5);  // 1.5 tiles of prologue + merge per CTA
+      if (cost < best - 1e-9) {
+        best = cost;
+        a.n_split = sp;
+      }
+    }
+  }
+  if (a.n_split > 1) {
+    const size_t nml = (size_t)nblk * a.n_split * 256 * sizeof(float2);
+    const size_t no = (size_t)nblk * a.n_split * 256 * p.d * sizeof(float);
+    void *cnt = nullptr, *data = nullptr;
+    if (workspace_get((size_t)nblk * sizeof(int), nml + no, &cnt, &data, stream) != SDPA_OK)
+      return cudaErrorMemoryAllocation;
+    a.ws_cnt = static_cast<int*>(cnt);
+    a.ws_ml = static_cast<float2*>(data);
+    a.ws_o = reinterpret_cast<float*>(static_cast<char*>(data) + nml);
+  }
+  dim3 grid((unsigned)(nqblk * a.n_split), (unsigned)p.Hq, (unsigned)p.B);
   if (!p.use_rel) {
     if (p.d == 64) return dispatch_mask<64, 128, 0, 3>(mk, a, grid, stream);
     return dispatch_mask<128, 128, 0, 2>(mk, a, grid, stream);

@@ -1,0 +1,348 @@
+// head_dim 16 kernels for the SAM mask decoder's attention shapes (mlx-examples
+// issue "segment_anything: fuse attention ...": the TwoWayTransformer's
+// Attention, the same matmul/softmax/matmul without a bias; candle PR "SDPA
+// with Relative Positional Embeddings": head_dim 16 support and a packed
+// vector kernel for it).  At head_dim 16 a 128-row tensor-core tile would sit
+// mostly idle and the work is a stream over Q/O or K/V, so both kernels run
+// on CUDA cores and are shaped for HBM bandwidth:
+//
+//  * small_d_kernel: one thread per query row (16 values of q, the running
+//    max/sum and a 16-wide accumulator in registers), 128 consecutive rows of
+//    one (batch, head) per CTA so Q and O move as fully coalesced 32-byte
+//    rows.  K/V of the kv head stream through shared memory in chunks as fp32
+//    and are read by every thread as broadcasts.  Used when there are many
+//    query rows (image->token: 4096 rows against 8 keys; self-attention).
+//
+//  * split_kv_kernel: few query rows against a long key axis (token->image: 8
+//    rows against 4096 keys).  The key axis of every (batch, head) is split
+//    over enough CTAs to cover the SMs; each CTA stages its K/V chunk in
+//    shared memory, one warp per query row runs the online softmax over the
+//    chunk (lanes stride the keys), and writes (m, l, unnormalised O) for its
+//    part.  The last CTA of a (batch, head) to finish, detected with an
+//    atomic ticket, merges the parts: O = sum_k 2^(m_k-M) O_k / sum_k 2^(m_k-M) l_k.
+//
+// Both take every mask kind and GQA; neither takes the rel-pos bias (the
+// exact kernel does).
+#include <math.h>
+
+#include "common.cuh"
+
+namespace sdpa {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int D16 = 16;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float* f) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// additive mask term (log2 units) or -inf for key j of row i; 0 when none
+__device__ __forceinline__ float mask_term(const Params& p, long long mrow, long long i, long long j) {
+  if (p.mask_kind == SDPA_MASK_ADD_FLOAT)
+    return __bfloat162float(static_cast<const __nv_bfloat16*>(p.mask)[mrow + j]) * kLog2e;
+  if (p.mask_kind == SDPA_MASK_BOOL)
+    return static_cast<const uint8_t*>(p.mask)[mrow + j] ? 0.f : -INFINITY;
+  if (p.mask_kind == SDPA_MASK_CAUSAL || p.mask_kind == SDPA_MASK_SLIDING) {
+    if (j > i + p.offset) return -INFINITY;
+    if (p.mask_kind == SDPA_MASK_SLIDING && j <= i + p.offset - p.window) return -INFINITY;
+  }
+  return 0.f;
+}
+
+// ------------------------------------------------------------------ small_d
+constexpr int kRowsPerCta = 128;
+constexpr int kKeyChunk = 128;
+
+__global__ void __launch_bounds__(kRowsPerCta) small_d_kernel(Params p) {
+  __shared__ float sk[kKeyChunk][D16];
+  __shared__ float sv[kKeyChunk][D16];
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.group;
+  const long long i = (long long)blockIdx.x * kRowsPerCta + threadIdx.x;
+  const bool valid = i < p.Tq;
+  const long long zq = (long long)b * p.Hq + h;
+  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (zq * p.Tq + (valid ? i : 0)) * D16;
+  float q[D16];
+  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
+  bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
+  const float sl = p.scale * kLog2e;
+#pragma unroll
+  for (int c = 0; c < D16; ++c) q[c] *= sl;
+
+  // key range shared by the CTA (causal / sliding), then per row
+  long long lo = 0, hi = p.Tkv;
+  if (p.mask_kind == SDPA_MASK_CAUSAL || p.mask_kind == SDPA_MASK_SLIDING) {
+    const long long first = (long long)blockIdx.x * kRowsPerCta;
+    const long long last = min(first + kRowsPerCta, (long long)p.Tq) - 1;
+    hi = min(hi, last + p.offset + 1);
+    if (p.mask_kind == SDPA_MASK_SLIDING) lo = max(0LL, first + p.offset - p.window + 1);
+  }
+  const bool elementwise = p.mask_kind != SDPA_MASK_NONE;
+  const long long mrow = (long long)b * p.msb + (long long)h * p.msh + i * p.msq;
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
+
+  float m = -INFINITY, l = 0.f, acc[D16];
+#pragma unroll
+  for (int c = 0; c < D16; ++c) acc[c] = 0.f;
+
+  for (long long j0 = lo; j0 < hi; j0 += kKeyChunk) {
+    const int n = (int)min((long long)kKeyChunk, hi - j0);
+    __syncthreads();
+    // stage the chunk: each thread moves one key's K row and V row (32 B each)
+    if (threadIdx.x < n) {
+      const long long j = j0 + threadIdx.x;
+      float f[D16];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * D16)), f);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * D16) + 1), f + 8);
+#pragma unroll
+      for (int c = 0; c < D16; ++c) sk[threadIdx.x][c] = f[c];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * D16)), f);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * D16) + 1), f + 8);
+#pragma unroll
+      for (int c = 0; c < D16; ++c) sv[threadIdx.x][c] = f[c];
+    }
+    __syncthreads();
+    if (!valid) continue;
+    for (int t = 0; t < n; ++t) {
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < D16; ++c) s = fmaf(q[c], sk[t][c], s);
+      if (elementwise) s += mask_term(p, mrow, i, j0 + t);
+      if (s == -INFINITY) continue;
+      if (s > m) {
+        const float corr = exp2f(m - s);  // 0 when m == -inf
+        l *= corr;
+#pragma unroll
+        for (int c = 0; c < D16; ++c) acc[c] *= corr;
+        m = s;
+      }
+      const float pj = exp2f(s - m);
+      l += pj;
+#pragma unroll
+      for (int c = 0; c < D16; ++c) acc[c] = fmaf(pj, sv[t][c], acc[c]);
+    }
+  }
+  if (!valid) return;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  uint4 o0, o1;
+  o0.x = pack2(acc[0] * inv, acc[1] * inv);
+  o0.y = pack2(acc[2] * inv, acc[3] * inv);
+  o0.z = pack2(acc[4] * inv, acc[5] * inv);
+  o0.w = pack2(acc[6] * inv, acc[7] * inv);
+  o1.x = pack2(acc[8] * inv, acc[9] * inv);
+  o1.y = pack2(acc[10] * inv, acc[11] * inv);
+  o1.z = pack2(acc[12] * inv, acc[13] * inv);
+  o1.w = pack2(acc[14] * inv, acc[15] * inv);
+  uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (zq * p.Tq + i) * D16);
+  orow[0] = o0;
+  orow[1] = o1;
+  if (p.lse) p.lse[zq * p.Tq + i] = l > 0.f ? m * kLn2 + logf(l) : -INFINITY;
+}
+
+// ------------------------------------------------------------------ split_kv
+constexpr int kSplitThreads = 256;  // 8 warps: one query row per warp at a time
+constexpr int kSplitChunk = 256;    // keys per CTA part (at most)
+
+struct SplitArgs {
+  Params p;
+  int nsplit;      // parts per (batch, head)
+  int chunk;       // keys per part
+  float* ws_o;     // [B*Hq][nsplit][Tq][16]
+  float2* ws_ml;   // [B*Hq][nsplit][Tq]  (m in log2 units, l)
+  int* ws_cnt;     // [B*Hq] tickets, zero between launches
+};
+
+__global__ void __launch_bounds__(kSplitThreads) split_kv_kernel(SplitArgs a) {
+  const Params& p = a.p;
+  __shared__ float sk[kSplitChunk][D16 + 1];
+  __shared__ float sv[kSplitChunk][D16 + 1];
+  __shared__ int s_last;
+  const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.group;
+  const long long zq = (long long)b * p.Hq + h;
+  const long long j0 = (long long)part * a.chunk;
+  const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
+  for (int t = threadIdx.x; t < n; t += kSplitThreads) {
+    float f[D16];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * D16)), f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * D16) + 1), f + 8);
+#pragma unroll
+    for (int c = 0; c < D16; ++c) sk[t][c] = f[c];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * D16)), f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * D16) + 1), f + 8);
+#pragma unroll
+    for (int c = 0; c < D16; ++c) sv[t][c] = f[c];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float sl = p.scale * kLog2e;
+  for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (zq * p.Tq + i) * D16;
+    float q[D16];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
+    const long long mrow = (long long)b * p.msb + (long long)h * p.msh + (long long)i * p.msq;
+    float m = -INFINITY, l = 0.f, acc[D16];
+#pragma unroll
+    for (int c = 0; c < D16; ++c) acc[c] = 0.f;
+    for (int t = lane; t < n; t += 32) {
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < D16; ++c) s = fmaf(q[c], sk[t][c], s);
+      s = s * sl + mask_term(p, mrow, i, j0 + t);
+      if (s == -INFINITY) continue;
+      if (s > m) {
+        const float corr = exp2f(m - s);
+        l *= corr;
+#pragma unroll
+        for (int c = 0; c < D16; ++c) acc[c] *= corr;
+        m = s;
+      }
+      const float pj = exp2f(s - m);
+      l += pj;
+#pragma unroll
+      for (int c = 0; c < D16; ++c) acc[c] = fmaf(pj, sv[t][c], acc[c]);
+    }
+    // combine the 32 lanes
+    float M = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    l *= w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+    for (int c = 0; c < D16; ++c) {
+      float x = acc[c] * w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      acc[c] = x;
+    }
+    if (lane == 0) {
+      const long long slot = (zq * a.nsplit + part) * p.Tq + i;
+      float4* dst = reinterpret_cast<float4*>(a.ws_o + slot * D16);
+#pragma unroll
+      for (int c = 0; c < D16; c += 4) __stcg(dst + c / 4, make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+      __stcg(a.ws_ml + slot, make_float2(M, l));
+    }
+  }
+  // the last part of this (batch, head) to finish merges all parts
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(a.ws_cnt + zq, 1) == a.nsplit - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
+    // lanes 0..15 own one output column each
+    float M = -INFINITY;
+    for (int k = lane; k < a.nsplit; k += 32) {
+      const float2 ml = __ldcg(a.ws_ml + (zq * a.nsplit + k) * p.Tq + i);
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f, num = 0.f;
+    for (int k = 0; k < a.nsplit; ++k) {
+      const long long slot = (zq * a.nsplit + k) * p.Tq + i;
+      const float2 ml = __ldcg(a.ws_ml + slot);
+      if (ml.y > 0.f) {
+        const float w = exp2f(ml.x - M);
+        den = fmaf(w, ml.y, den);
+        if (lane < D16) num = fmaf(w, __ldcg(a.ws_o + slot * D16 + lane), num);
+      }
+    }
+    const float val = den > 0.f ? num / den : 0.f;
+    const float nb = __shfl_down_sync(0xffffffffu, val, 1);
+    if (lane < D16 && (lane & 1) == 0) {
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + (zq * p.Tq + i) * D16;
+      *reinterpret_cast<uint32_t*>(orow + lane) = pack2(val, nb);
+    }
+    if (lane == 0 && p.lse) p.lse[zq * p.Tq + i] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
+  }
+  if (threadIdx.x == 0) a.ws_cnt[zq] = 0;  // ready for the next launch
+}
+
+}  // namespace
+
+int small_d_check(const Params& p, sdpa_dtype_t dtype) {
+  if (dtype != SDPA_BF16 || p.d != 16) return SDPA_ERR_UNSUPPORTED;
+  if (p.use_rel) return SDPA_ERR_UNSUPPORTED;
+  if (p.B > 65535 || p.Hq > 65535) return SDPA_ERR_UNSUPPORTED;
+  const uintptr_t m = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
+                      reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.out);
+  if (m & 15) return SDPA_ERR_MISALIGNED;
+  return SDPA_OK;
+}
+
+cudaError_t launch_small_d(const Params& p, cudaStream_t stream) {
+  dim3 grid((unsigned)((p.Tq + kRowsPerCta - 1) / kRowsPerCta), (unsigned)p.Hq, (unsigned)p.B);
+  small_d_kernel<<<grid, kRowsPerCta, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+int split_kv_check(const Params& p, sdpa_dtype_t dtype) { return small_d_check(p, dtype); }
+
+// Parts per (batch, head): enough CTAs for two per SM, parts of at most
+// kSplitChunk keys.
+static void split_shape(const Params& p, int* nsplit, int* chunk) {
+  const long long bh = (long long)p.B * p.Hq;
+  const long long want = (2LL * num_sms() + bh - 1) / bh;
+  long long ns = max(1LL, min(want, (long long)(p.Tkv + 31) / 32));
+  long long ch = (p.Tkv + ns - 1) / ns;
+  if (ch > kSplitChunk) {
+    ch = kSplitChunk;
+    ns = (p.Tkv + ch - 1) / ch;
+  }
+  *nsplit = (int)ns;
+  *chunk = (int)ch;
+}
+
+void split_kv_workspace_bytes(const Params& p, size_t* cnt_bytes, size_t* data_bytes) {
+  int ns, ch;
+  split_shape(p, &ns, &ch);
+  const long long bh = (long long)p.B * p.Hq;
+  const size_t nml = (size_t)bh * ns * p.Tq * sizeof(float2);
+  const size_t no = (size_t)bh * ns * p.Tq * D16 * sizeof(float);
+  *cnt_bytes = (size_t)bh * sizeof(int);
+  *data_bytes = ((nml + 255) & ~size_t(255)) + no;
+}
+
+cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream_t stream) {
+  SplitArgs a;
+  a.p = p;
+  split_shape(p, &a.nsplit, &a.chunk);
+  const long long bh = (long long)p.B * p.Hq;
+  const size_t nml = (size_t)bh * a.nsplit * p.Tq * sizeof(float2);
+  a.ws_cnt = cnt;
+  a.ws_ml = static_cast<float2*>(data);
+  a.ws_o = reinterpret_cast<float*>(static_cast<char*>(data) + ((nml + 255) & ~size_t(255)));
+  dim3 grid((unsigned)a.nsplit, (unsigned)p.Hq, (unsigned)p.B);
+  split_kv_kernel<<<grid, kSplitThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_kv(const Params& p, cudaStream_t stream) {
+  size_t cb = 0, db = 0;
+  split_kv_workspace_bytes(p, &cb, &db);
+  void *cnt = nullptr, *data = nullptr;
+  if (workspace_get(cb, db, &cnt, &data, stream) != SDPA_OK) return cudaErrorMemoryAllocation;
+  return launch_split_kv_ws(p, static_cast<int*>(cnt), data, stream);
+}
+
+}  // namespace sdpa

@@ -57,6 +57,16 @@ CASES = [
     S_("bool_bf16_d128_bcast", BF16, 1, 4, 4, 130, 128, 128, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.9,
        mask_heads=1, seed=25),
     S_("mqa_bf16_d128", BF16, 2, 8, 1, 200, 256, 128, seed=26),
+    # head_dim 16: mask-decoder shapes, reduced, with every mask kind and GQA
+    S_("d16_cross_short_q", BF16, 2, 4, 2, 9, 1500, 16, seed=40),
+    S_("d16_cross_short_kv", BF16, 2, 4, 4, 700, 7, 16, seed=41),
+    S_("d16_causal_gqa", BF16, 1, 4, 2, 300, 300, 16, mask_kind=W.MASK_CAUSAL, offset=3, seed=42),
+    S_("d16_float_mask", BF16, 2, 2, 2, 40, 1100, 16, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.3, mask_heads=2, seed=43),
+    S_("d16_bool_mask", BF16, 1, 2, 1, 130, 333, 16, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.6,
+       mask_heads=1, seed=44),
+    S_("d16_sliding_long_kv", BF16, 1, 2, 2, 16, 3000, 16, mask_kind=W.MASK_SLIDING, window=700, offset=2000,
+       seed=45),
     # rel-pos shapes the tensor-core path specialises (key-grid width 14/16/32/64)
     S_("relpos_bf16_d64_12x16", BF16, 2, 3, 3, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5, seed=27),
     S_("relpos_bf16_d64_8x32", BF16, 1, 4, 2, 256, 256, 64, q_hw=(8, 32), k_hw=(8, 32), rel_std=0.5, seed=28),
@@ -95,10 +105,8 @@ def applicable(path: str, sp: W.Spec) -> bool:
                     and ((2 * max(kh, kw) - 1) + 15) // 16 * 16 <= bn
                     and sp.mask_kind in (W.MASK_NONE, W.MASK_CAUSAL, W.MASK_SLIDING))
         return True
-    if path == "small_d":
-        return sp.d == 16
-    if path == "split_kv":
-        return not sp.rel and sp.mask_kind == W.MASK_NONE
+    if path in ("small_d", "split_kv"):
+        return sp.d == 16 and not sp.rel
     return False
 
 
@@ -107,7 +115,7 @@ def _implemented(path):
     return path in _BUILT
 
 
-_BUILT = {"exact", "tcgen05"}
+_BUILT = {"exact", "tcgen05", "small_d", "split_kv"}
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -125,7 +133,7 @@ def test_parity(sp, path):
     assert np.max(np.abs(got[fin] - ref.lse[fin])) < 2e-3, "lse"
 
 
-@pytest.mark.parametrize("path", ["exact", "tcgen05"])
+@pytest.mark.parametrize("path", ["exact", "tcgen05", "small_d", "split_kv"])
 def test_edge_cases(path):
     _edge_cases(path)
 
@@ -133,35 +141,36 @@ def test_edge_cases(path):
 def _edge_cases(path):
     import attention_sdpa_fwd_b200 as S
     dev = "cuda"
+    d = 16 if path in ("small_d", "split_kv") else 64
     if path == "exact":
         # Tkv = 0: every row sees nothing -> zeros, lse = -inf
-        q = torch.randn(1, 2, 5, 64, device=dev, dtype=BF16)
-        e = torch.empty(1, 2, 0, 64, device=dev, dtype=BF16)
+        q = torch.randn(1, 2, 5, d, device=dev, dtype=BF16)
+        e = torch.empty(1, 2, 0, d, device=dev, dtype=BF16)
         lse = torch.zeros(1, 2, 5, device=dev)
         out = torch.full_like(q, 7.0)
         S.sdpa(q, e, e, 0.1, out=out, lse=lse, path=path)
         torch.cuda.synchronize()
         assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
     # causal with a large negative offset: no row sees a key -> zeros, lse = -inf
-    q = torch.randn(1, 2, 300, 64, device=dev, dtype=BF16)
+    q = torch.randn(1, 2, 300, d, device=dev, dtype=BF16)
     lse = torch.zeros(1, 2, 300, device=dev)
     out = torch.full_like(q, 7.0)
     S.sdpa(q, q, q, 0.1, mask_kind=S.MASK_CAUSAL, offset=-400, out=out, lse=lse, path=path)
     torch.cuda.synchronize()
     assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
     # B = 0: nothing to do
-    z = torch.empty(0, 2, 5, 64, device=dev, dtype=BF16)
+    z = torch.empty(0, 2, 5, d, device=dev, dtype=BF16)
     S.sdpa(z, z, z, 0.1, path=path)
     # Tq = Tkv = 1: output is v
-    q1 = torch.randn(2, 2, 1, 64, device=dev, dtype=BF16)
-    k1 = torch.randn(2, 2, 1, 64, device=dev, dtype=BF16)
-    v1 = torch.randn(2, 2, 1, 64, device=dev, dtype=BF16)
+    q1 = torch.randn(2, 2, 1, d, device=dev, dtype=BF16)
+    k1 = torch.randn(2, 2, 1, d, device=dev, dtype=BF16)
+    v1 = torch.randn(2, 2, 1, d, device=dev, dtype=BF16)
     o1 = S.sdpa(q1, k1, v1, path=path)
     torch.cuda.synchronize()
     assert torch.equal(o1, v1)
     # fully masked rows (bool) -> zeros
-    q2 = torch.randn(1, 1, 130, 64, device=dev, dtype=BF16)
-    k2 = torch.randn(1, 1, 144, 64, device=dev, dtype=BF16)
+    q2 = torch.randn(1, 1, 130, d, device=dev, dtype=BF16)
+    k2 = torch.randn(1, 1, 144, d, device=dev, dtype=BF16)
     keep = torch.ones(1, 1, 130, 144, device=dev, dtype=torch.uint8)
     keep[0, 0, 3] = 0
     keep[0, 0, 129] = 0
