@@ -51,6 +51,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank floats over all ranks (identity at one rank)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate_throughput(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job TFLOP/s: every rank runs its own problem (weak scaling), the
+    job takes as long as the slowest rank."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -307,20 +322,13 @@ def run_ours(args):
 
     ms = r["total_ms"] / args.steps
     launch_avg = sum(r["launch_ms"]) / len(r["launch_ms"])
-    # max over ranks
-    if ws > 1:
-        t = torch.tensor([ms, launch_avg], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, launch_avg = float(t[0]), float(t[1])
+    ms, launch_avg = max_over_ranks([ms, launch_avg], device)
     flops = spec.flops()
-    value = ws * flops / (ms * 1e-3) / 1e12
+    value = aggregate_throughput(flops, ms, ws)
 
     e2e_ms, h2d, d2h = time_e2e(S, spec, device, max(3, min(args.steps, 20)), 2)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e = ws * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms, = max_over_ranks([e2e_ms], device)
+    e2e = aggregate_throughput(flops, e2e_ms, ws)
 
     per_config = {}
     if args.per_config and rank == 0:
