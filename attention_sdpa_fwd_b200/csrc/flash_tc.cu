@@ -57,6 +57,12 @@ constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-po
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Pairs of score columns whose index satisfies (i & kEmuMask) == kEmuMask take
+// 2^y on the FMA pipe (negative: every exponential on the MUFU unit).
+#ifndef SDPA_EMU_MASK
+#define SDPA_EMU_MASK -1
+#endif
+constexpr int kEmuMask = SDPA_EMU_MASK;
 
 enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3 };
 
@@ -97,6 +103,31 @@ struct Layout {
   static_assert(kAlloc <= 232448, "shared memory budget");
   static_assert(KW == 0 || (BN % (KW > 0 ? KW : 1) == 0), "key tile must hold whole key-grid rows");
 };
+
+// 2^y for a pair, on the FMA pipe: Cody-Waite reduction y = n + f with
+// n = round(y) (the magic-number add leaves n in the low mantissa bits of t),
+// f in [-1/2, 1/2]; 2^f by the degree-3 minimax polynomial of
+// fit_exp2_poly.py (max relative error 7.5e-5, well under bf16's 2^-9); 2^n
+// added straight into the exponent field.  y is clamped at -125 so the result
+// stays a normal number (callers only use it where no score is -inf).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t y2) {
+  float y0, y1;
+  f2_split(y2, y0, y1);
+  y2 = f2(fmaxf(y0, -125.f), fmaxf(y1, -125.f));
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t t2 = f2_add(y2, f2(kMagic, kMagic));
+  const uint64_t n2 = f2_add(t2, f2(-kMagic, -kMagic));
+  const uint64_t fr = f2_fma(n2, f2(-1.f, -1.f), y2);
+  uint64_t p2 = f2_fma(fr, f2(5.517166906e-02f, 5.517166906e-02f), f2(2.426111222e-01f, 2.426111222e-01f));
+  p2 = f2_fma(p2, fr, f2(6.932609855e-01f, 6.932609855e-01f));
+  p2 = f2_fma(p2, fr, f2(9.999280735e-01f, 9.999280735e-01f));
+  float p0, p1, t0, t1;
+  f2_split(p2, p0, p1);
+  f2_split(t2, t0, t1);
+  const uint32_t r0 = __float_as_uint(t0) * 8388608u + __float_as_uint(p0);  // += n << 23
+  const uint32_t r1 = __float_as_uint(t1) * 8388608u + __float_as_uint(p1);
+  return f2u(r0, r1);
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -619,8 +650,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         }
       }
 
-      // p = 2^(x + goff - m), packed to bf16 pairs and written to P in TMEM
+      // p = 2^(x + goff - m), packed to bf16 pairs and written to P in TMEM.
+      // Some pairs take 2^y on the FMA pipe instead of the MUFU unit (only on
+      // tiles that hold no -inf: the polynomial path cannot return an exact 0).
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const bool emu = kEmuMask >= 0 && (MASK == TC_NONE) && (j0 + BN <= args.Tkv);
       uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -629,10 +663,16 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         for (int i = 0; i < 8; ++i) {
           const int c = c0 + 2 * i;
           const float nmo = goff[c / GW] - m_use;
-          float lo, hi;
-          f2_split(f2_add(x2[c / 2], f2(nmo, nmo)), lo, hi);
-          const float p0 = ex2_approx(lo);
-          const float p1 = ex2_approx(hi);
+          const uint64_t y2 = f2_add(x2[c / 2], f2(nmo, nmo));
+          float p0, p1;
+          if (kEmuMask >= 0 && emu && ((c / 2) & kEmuMask) == kEmuMask) {
+            f2_split(exp2_poly2(y2), p0, p1);
+          } else {
+            float lo, hi;
+            f2_split(y2, lo, hi);
+            p0 = ex2_approx(lo);
+            p1 = ex2_approx(hi);
+          }
           sum2[i & 1] = f2_add(sum2[i & 1], f2(p0, p1));
           r8[i] = pack_bf16x2(p0, p1);
         }
@@ -895,7 +935,9 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
     double best = 1e30;
     for (int sp = 1; sp <= 8 && sp <= nt; ++sp) {
       const double waves = (double)((nblk * sp + nsm - 1) / nsm);
-      const double cost = waves * ((nt + sp - 1) / sp + 1.5);  // 1.5 tiles of prologue + merge per CTA
+      // per-CTA fixed cost (prologue, partial write-out, merge) measured at
+      // about 16 key tiles' worth on B200
+      const double cost = waves * ((nt + sp - 1) / sp + 16.0);
       if (cost < best - 1e-9) {
         best = cost;
         a.n_split = sp;
