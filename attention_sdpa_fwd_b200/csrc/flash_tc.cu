@@ -216,6 +216,19 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   tc_fence_after();
   const uint32_t tbase = *tslot;
   volatile int* abort_v = abort_flag;
+  constexpr bool kWarpIssue = !kPSep;
+  auto mma_ss_x = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    if constexpr (kWarpIssue) mma_ss_w(d, a, b, id, acc); else mma_ss(d, a, b, id, acc);
+  };
+  auto mma_ts_x = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    if constexpr (kWarpIssue) mma_ts_w(d, a, b, id, acc); else mma_ts(d, a, b, id, acc);
+  };
+  auto mma_commit_x = [](uint64_t* bar) {
+    if constexpr (kWarpIssue) mma_commit_w(bar); else mma_commit(bar);
+  };
+  auto wait_x = [](bool v) {
+    if constexpr (kWarpIssue) return __all_sync(0xffffffffu, v); else return v;
+  };
 
   // Register split: the producer/MMA warpgroup gives registers to the two
   // softmax warpgroups (3 x 128 x 168 at launch = 2 x 128 x 232 + 128 x 40).
@@ -283,7 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    // At head_dim 128 the whole warp runs the loop and one elected lane issues
+    // each instruction (measured faster there); at 64 lane 0 runs it alone.
+    if ((kWarpIssue || lane == 0) && n_tiles > 0) {
       constexpr uint32_t id_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t id_pv = idesc_bf16_f32(128, D, false, true);
       // Descriptors are built once; a byte offset inside shared memory is added
@@ -291,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       const uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dv = sdesc_sw128(smem_u32(sV), BN * 128, 1024);
-      bool ok = mbar_wait(q_full, 0, abort_v, args.err);
+      bool ok = wait_x(mbar_wait(q_full, 0, abort_v, args.err));
       auto qk = [&](int t, int s) {
         const uint64_t a0 = dq + (uint64_t)((t * L::kQBytes) >> 4);
         const uint64_t b0 = dk + (uint64_t)((s * L::kKVBytes) >> 4);
@@ -300,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = ((kk >> 2) * (kRowsPerTile * 128) + (kk & 3) * 32) >> 4;
           const uint32_t bo = ((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4;
-          mma_ss(d_tm, a0 + ao, b0 + bo, id_qk, kk > 0);
+          mma_ss_x(d_tm, a0 + ao, b0 + bo, id_qk, kk > 0);
         }
       };
       auto pv = [&](int t, int s, bool first) {
@@ -309,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         const uint32_t a_tm = kPSep ? tbase + 384 + t * 64 : tbase + t * 128;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(d_tm, a_tm + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (!first) || kk > 0);
+          mma_ts_x(d_tm, a_tm + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (!first) || kk > 0);
       };
       if (ok && KW > 0) {
         // rel projections: Ph_t -> cols [256t, 256t+rel_n), Pw_t -> [256t+128, 256t+128+rel_n)
@@ -321,20 +336,20 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           for (int w = 0; w < 2; ++w)
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tbase + t * 256 + w * 128, dq + (uint64_t)((t * L::kQBytes + kk * 32) >> 4),
+              mma_ss_x(tbase + t * 256 + w * 128, dq + (uint64_t)((t * L::kQBytes + kk * 32) >> 4),
                      (w == 0 ? drh : drw) + (uint64_t)((kk * 32) >> 4), id_rel, kk > 0);
-        mma_commit(rel_mma);
-        ok = mbar_wait(rel_read, 0, abort_v, args.err);
+        mma_commit_x(rel_mma);
+        ok = wait_x(mbar_wait(rel_read, 0, abort_v, args.err));
       }
       // prologue: S_A(0), S_B(0)
-      if (ok) ok = mbar_wait(&k_full[0], 0, abort_v, args.err);
+      if (ok) ok = wait_x(mbar_wait(&k_full[0], 0, abort_v, args.err));
       if (ok) {
         tc_fence_after();
         qk(0, 0);
-        mma_commit(&s_full[0]);
+        mma_commit_x(&s_full[0]);
         qk(1, 0);
-        mma_commit(&s_full[1]);
-        mma_commit(&k_empty[0]);
+        mma_commit_x(&s_full[1]);
+        mma_commit_x(&k_empty[0]);
       }
       if constexpr (kPSep) {
         // A and B alternate: S_A(j+1), O_A += P_A(j).V_j, S_B(j+1), O_B += P_B(j).V_j
@@ -343,68 +358,68 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           const bool more = jj + 1 < n_tiles;
           const int s1 = (jj + 1) % NS;
           if (more) {
-            ok = mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err);
-            if (ok) ok = mbar_wait(&s_free[0], jj & 1, abort_v, args.err);
+            ok = wait_x(mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err));
+            if (ok) ok = wait_x(mbar_wait(&s_free[0], jj & 1, abort_v, args.err));
             if (!ok) break;
             tc_fence_after();
             qk(0, s1);
-            mma_commit(&s_full[0]);
+            mma_commit_x(&s_full[0]);
           }
-          ok = mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err);
-          if (ok) ok = mbar_wait(&p_full[0], jj & 1, abort_v, args.err);
+          ok = wait_x(mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err));
+          if (ok) ok = wait_x(mbar_wait(&p_full[0], jj & 1, abort_v, args.err));
           if (!ok) break;
           tc_fence_after();
           pv(0, s, jj == 0);
-          mma_commit(&o_ready[0]);
+          mma_commit_x(&o_ready[0]);
           if (more) {
-            ok = mbar_wait(&s_free[1], jj & 1, abort_v, args.err);
+            ok = wait_x(mbar_wait(&s_free[1], jj & 1, abort_v, args.err));
             if (!ok) break;
             tc_fence_after();
             qk(1, s1);
-            mma_commit(&s_full[1]);
-            mma_commit(&k_empty[s1]);
+            mma_commit_x(&s_full[1]);
+            mma_commit_x(&k_empty[s1]);
           }
-          ok = mbar_wait(&p_full[1], jj & 1, abort_v, args.err);
+          ok = wait_x(mbar_wait(&p_full[1], jj & 1, abort_v, args.err));
           if (!ok) break;
           tc_fence_after();
           pv(1, s, jj == 0);
-          mma_commit(&o_ready[1]);
-          mma_commit(&v_empty[s]);
+          mma_commit_x(&o_ready[1]);
+          mma_commit_x(&v_empty[s]);
         }
       } else {
         for (int jj = 0; jj < n_tiles && ok; ++jj) {
           const int s = jj % NS;
-          ok = mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err);
+          ok = wait_x(mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err));
           if (!ok) break;
           // tile A: O_A += P_A V_j, then S_A(j+1)
-          ok = mbar_wait(&p_full[0], jj & 1, abort_v, args.err);
+          ok = wait_x(mbar_wait(&p_full[0], jj & 1, abort_v, args.err));
           if (!ok) break;
           tc_fence_after();
           pv(0, s, jj == 0);
           const bool more = jj + 1 < n_tiles;
           const int s1 = (jj + 1) % NS;
           if (more) {
-            ok = mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err);
+            ok = wait_x(mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err));
             if (!ok) break;
             tc_fence_after();
             qk(0, s1);
-            mma_commit(&s_full[0]);
+            mma_commit_x(&s_full[0]);
           }
           // tile B: O_B += P_B V_j, release V_j, then S_B(j+1) and release K_{j+1}
-          ok = mbar_wait(&p_full[1], jj & 1, abort_v, args.err);
+          ok = wait_x(mbar_wait(&p_full[1], jj & 1, abort_v, args.err));
           if (!ok) break;
           tc_fence_after();
           pv(1, s, jj == 0);
-          mma_commit(&v_empty[s]);
+          mma_commit_x(&v_empty[s]);
           if (more) {
             qk(1, s1);
-            mma_commit(&s_full[1]);
-            mma_commit(&k_empty[s1]);
+            mma_commit_x(&s_full[1]);
+            mma_commit_x(&k_empty[s1]);
           }
         }
       }
-      mma_commit(&o_done[0]);
-      mma_commit(&o_done[1]);
+      mma_commit_x(&o_done[0]);
+      mma_commit_x(&o_done[1]);
     }
   }
   } else {
