@@ -26,7 +26,7 @@ STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
           -6: "SDPA_ERR_CAPACITY"}
 
 # Every symbol include/sdpa.h declares.
-EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_select_path", "sdpa_fwd_host",
+EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_select_path", "sdpa_fwd_host", "sdpa_fwd_split_kv_static",
            "sdpa_last_device_error", "sdpa_strerror", "sdpa_version")
 
 
@@ -58,11 +58,12 @@ def lib():
         L.sdpa_fwd_ex.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
         L.sdpa_fwd_host.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
         L.sdpa_select_path.argtypes = _COMMON + [_i32, _vp, _vp, _vp, _vp, _vp]
+        L.sdpa_fwd_split_kv_static.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp]
         L.sdpa_last_device_error.argtypes = [_vp]
         L.sdpa_strerror.argtypes = [_i32]
         L.sdpa_strerror.restype = ctypes.c_char_p
         for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_host", "sdpa_select_path",
-                     "sdpa_last_device_error", "sdpa_version"):
+                     "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_version"):
             getattr(L, name).restype = _i32
         _lib = L
     return _lib
@@ -97,6 +98,12 @@ def sdpa_select_path(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, mask_kind, mas
                      rel_pos_h, rel_pos_w, q_hw, k_hw) -> int:
     return lib().sdpa_select_path(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, mask_kind, mask_ptr,
                                   rel_pos_h, rel_pos_w, _hw(q_hw), _hw(k_hw))
+
+
+def sdpa_fwd_split_kv_static(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                             lse, stream) -> int:
+    return lib().sdpa_fwd_split_kv_static(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind,
+                                          mask_ptr, lse, stream)
 
 
 def sdpa_last_device_error(stream) -> int:

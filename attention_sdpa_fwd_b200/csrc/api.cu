@@ -359,6 +359,21 @@ extern "C" int sdpa_fwd_host(const void* q, const void* k, const void* v, void* 
   return SDPA_OK;
 }
 
+extern "C" int sdpa_fwd_split_kv_static(const void* q, const void* k, const void* v, void* out,
+                                        sdpa_dtype_t dtype, int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                                        float scale, int mask_kind, const void* mask_ptr, float* lse,
+                                        cudaStream_t stream) {
+  Problem pr;
+  int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr, nullptr,
+                         nullptr, nullptr, nullptr, lse, &pr);
+  if (rc != SDPA_OK) return rc;
+  if (pr.empty_out) return SDPA_OK;
+  Params p = pr.p;
+  p.err = error_word_ptr();
+  if (p.err == nullptr) return SDPA_ERR_CUDA;
+  return split_kv_static(p, pr.dtype, stream);
+}
+
 extern "C" int sdpa_last_device_error(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return SDPA_ERR_CUDA;
   int* w = error_word_ptr();

@@ -74,6 +74,8 @@ cudaError_t launch_split_kv(const Params& p, cudaStream_t stream);
 // zero at launch, and partial results) and the launch on given scratch
 void split_kv_workspace_bytes(const Params& p, size_t* cnt_bytes, size_t* data_bytes);
 cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream_t stream);
+// split-KV on the fixed-size static scratch (no allocation); an sdpa_status
+int split_kv_static(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
 int num_sms();
 cudaError_t launch_tc(const Params& p, cudaStream_t stream);
 

@@ -99,7 +99,7 @@ typedef enum {
   SDPA_PATH_EXACT = 1,     /* CUDA-core FFMA online softmax; every feature, fp32 and bf16 */
   SDPA_PATH_TCGEN05 = 2,   /* TMA + tcgen05/TMEM flash kernel; bf16, d in {64,128} */
   SDPA_PATH_SMALL_D = 3,   /* packed d=16 kernel, one query row per thread; bf16 */
-  SDPA_PATH_SPLIT_KV = 4   /* split-KV with in-kernel merge, short Tq / long Tkv; bf16, d=16..128 */
+  SDPA_PATH_SPLIT_KV = 4   /* split-KV with in-kernel merge, short Tq / long Tkv; bf16, d=16 */
 } sdpa_path_t;
 
 /*
@@ -173,6 +173,30 @@ int sdpa_fwd_host(const void* q, const void* k, const void* v, void* out, sdpa_d
                   const void* rel_pos_h, const void* rel_pos_w,
                   const int* q_hw, const int* k_hw,
                   int path, cudaStream_t stream);
+
+/*
+ * sdpa_fwd_split_kv_static -- the split-KV forward (bf16, head_dim 16, every
+ * mask kind, no rel-pos) for callers that cannot allocate device memory during
+ * a call, e.g. code running under a memory pool it does not own or whose
+ * start-up already reserved all the memory it may use.  (The pages have no
+ * counterpart; this is an entry point of the library, not of the method.)
+ *
+ * It allocates nothing: its scratch is a fixed 4 MiB device array inside the
+ * library (64 KiB of tickets, one per (batch, head), and the partial results),
+ * held by every device that loads the library until the process exits.
+ * Problems whose scratch does not fit return SDPA_ERR_CAPACITY; an
+ * unsupported shape returns SDPA_ERR_UNSUPPORTED.  q, k, v, out (and lse, may
+ * be NULL) are caller-owned device pointers exactly as for sdpa_fwd_ex.
+ *
+ * The first call on a device looks up the array's device address; make that
+ * first call before capturing a stream into a graph.  Every call on a device
+ * shares the array and leaves its contents behind: calls whose kernels may
+ * overlap on the GPU (different streams without ordering between them) race
+ * on it and must not be issued; calls on one stream are ordered and safe.
+ */
+int sdpa_fwd_split_kv_static(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
+                             int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
+                             int mask_kind, const void* mask_ptr, float* lse, cudaStream_t stream);
 
 /* Synchronises `stream`, then returns and clears the device error word of the
    current device: SDPA_OK, or SDPA_ERR_TIMEOUT when a kernel gave up a bounded
