@@ -144,7 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   constexpr bool kRwInSmem = KW >= 32;  // large key-grid width: rel_w re-read per tile
   constexpr int kRwSwz = KW >= 64 ? 15 : 7;  // float4-index XOR swizzle of those rows (conflict-free)
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // offset from smem_raw (not a cast through an integer) so that the
+  // compiler keeps the shared address space and emits shared loads
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem + L::oQ;
   uint8_t* sK = smem + L::oK;
   uint8_t* sV = smem + L::oV;
