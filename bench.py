@@ -74,35 +74,84 @@ def dist_env():
 
 
 # ---------------------------------------------------------------------------
-# clocks sampler (nvidia-smi during the timed region)
+# clocks sampler (NVML read-only queries during the timed region)
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """Polls the SM clock and the active clock-event reasons every ~1 ms on a
+    background thread (NVML reads only; no setting is touched).  The timed
+    region of one bench step is short (well under a second), so a 1 ms cadence
+    is what puts samples inside it.  Falls back to ``nvidia-smi -lms 50``."""
+    REASONS = (("hw_slowdown", "HwSlowdown"), ("hw_thermal_slowdown", "HwThermalSlowdown"),
+               ("sw_thermal_slowdown", "SwThermalSlowdown"), ("sw_power_cap", "SwPowerCap"),
+               ("hw_power_brake", "HwPowerBrakeSlowdown"))
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
-        self.samples = []
-        self.proc = None
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []          # (time, sm_mhz, max_mhz, [reason names])
+        self.source = "none"
+        self._stop = threading.Event()
         self.thread = None
+        self.proc = None
+
+    def _nvml_handle(self, nv):
+        try:
+            pr = torch.cuda.get_device_properties(self.cuda_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._nvml_handle(nv)
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            bits = [(name, getattr(nv, "nvmlClocksEventReason" + suffix, 0)) for name, suffix in self.REASONS]
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        r = get_reasons(h)
+                    except Exception:
+                        break
+                    self.samples.append((time.time(), mhz, mx, [n for n, b in bits if b and (r & b)]))
+                    time.sleep(0.001)
+            self.source = "nvml"
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.cuda_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            return
+        self.source = "nvidia-smi"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+        def read():
+            for line in self.proc.stdout:
+                parts = [x.strip() for x in line.split(",")]
+                try:
+                    self.samples.append((time.time(), float(parts[1]), float(parts[2]),
+                                         [n for n, v in zip(names, parts[5:9]) if v.lower() == "active"]))
+                except (ValueError, IndexError):
+                    continue
+        self.thread = threading.Thread(target=read, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.samples.append((time.time(), line.strip()))
-
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -113,28 +162,16 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self, t0: float, t1: float):
-        rows = []
-        for ts, line in self.samples:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((ts, float(parts[1]), float(parts[2]), parts))
-            except ValueError:
-                continue
+        rows = list(self.samples)
         inside = [r for r in rows if t0 <= r[0] <= t1]
         used = inside if inside else sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
         if not used:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "source": self.source}
         mhz = sorted(r[1] for r in used)
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in used:
-            for n, v in zip(names, r[3][5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(r[2] for r in used),
-                "reasons": sorted(reasons), "samples": len(used), "samples_in_window": len(inside)}
+        reasons = sorted({n for r in used for n in r[3]})
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(r[2] for r in used), "reasons": reasons,
+                "samples": len(used), "samples_in_window": len(inside), "source": self.source}
 
 
 # ---------------------------------------------------------------------------
@@ -297,6 +334,29 @@ def cpu_oracle_sample(spec: W.Spec, budget_s: float = 12.0):
                        f"(fp64, {sec:.1f} s)", seconds=sec)
 
 
+def run_profile_launches(args):
+    """Untimed launches for an ncu capture: one input set of the workload with
+    its batch scaled by --batch-mult (so a small case can still exceed L2),
+    --profile-launches calls, then the device error word.  Prints one status
+    line, not a bench line."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    import attention_sdpa_fwd_b200 as S
+    S.lib()
+    spec = W.SPECS[args.workload]
+    spec = W.scaled(spec, B=spec.B * args.batch_mult)
+    st = make_device_sets(spec, device, 1, seed_base=spec.seed)[0]
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.profile_launches):
+        launch(S, spec, st, stream, 0)
+    torch.cuda.synchronize(device)
+    rc = S.sdpa_last_device_error(stream.cuda_stream)
+    print(f"profile launches: {spec.name} B={spec.B} x{args.profile_launches} "
+          f"({spec.bytes() / 1e6:.1f} MB per launch) device error {rc}", flush=True)
+    if rc != 0:
+        sys.exit(1)
+
+
 def run_ours(args):
     ws, rank, local = dist_env()
     if ws > 1:
@@ -423,10 +483,16 @@ def main():
     ap.add_argument("--per-config", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--profile-launches", type=int, default=0,
+                    help="only run this many untimed launches (for ncu) and exit")
+    ap.add_argument("--batch-mult", type=int, default=1,
+                    help="with --profile-launches: multiply the workload's batch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_launches > 0:
+        run_profile_launches(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
