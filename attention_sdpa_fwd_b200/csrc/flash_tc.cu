@@ -34,6 +34,8 @@
 // and rel_w[i, kw] = Pw[i, qw - kw + Kw - 1] (times log2 e) into shared
 // memory, from where the loop adds them to the scores before the row max.
 #include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -48,6 +50,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
+constexpr int kMaxSplit = 8;  // parts one unit's key range may be split into
 constexpr int kRegsLaunch = 168;   // registers per thread the kernel is launched with
 constexpr int kRegsSoftmax = 224;  // after setmaxnreg, softmax warpgroups
 constexpr int kRegsOther = 56;     // after setmaxnreg, producer / MMA warpgroup
@@ -79,10 +82,18 @@ struct TcArgs {
   int qw_n, kh_n, kw_n;
   int rel_n;  // rows of the padded rel tables (multiple of 16, <= 128)
   int mask_vec;  // mask rows allow 16-byte vector loads
-  int n_split;   // CTAs sharing one 256-row query block (key range split); 1 = no split
-  float* ws_o;   // [blocks][n_split][256][D] unnormalised partial outputs   (n_split > 1)
-  float2* ws_ml; // [blocks][n_split][256] (running max in log2 units, sum)   (n_split > 1)
-  int* ws_cnt;   // [blocks] arrival counters, zero between launches         (n_split > 1)
+  // Work decomposition over a 1-D grid.  A unit is one 256-row query block of
+  // one (batch, head); units are numbered with the query block fastest.  CTAs
+  // [0, n_full) each take unit blockIdx.x whole; after them every n_split
+  // consecutive CTAs share the key range of one further unit (n_full + i),
+  // each taking one contiguous part, merged in-kernel by the last to finish.
+  int nqblk;     // query blocks per (batch, head)
+  int n_full;    // units taken whole, first in launch order
+  int n_split;   // parts per split unit (1 = no split units)
+  int reverse_q; // take query blocks last-first (causal: the longest rows start first)
+  float* ws_o;   // [split units][n_split][D/4][256] float4: unnormalised partial outputs
+  float2* ws_ml; // [split units][n_split][256] (running max in log2 units, sum)
+  int* ws_cnt;   // [split units] arrival counters, zero between launches
   int* err;
 };
 
@@ -171,11 +182,19 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int nsplit = args.n_split;
-  const int qblk = blockIdx.x / nsplit;
-  const int sidx = blockIdx.x - qblk * nsplit;  // which part of the key range this CTA takes
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  int unit, sidx = 0, nsplit = 1;  // sidx: which part of the unit's key range this CTA takes
+  if ((int)blockIdx.x < args.n_full) {
+    unit = blockIdx.x;
+  } else {
+    const int i = blockIdx.x - args.n_full;
+    nsplit = args.n_split;
+    unit = args.n_full + i / nsplit;
+    sidx = i - (i / nsplit) * nsplit;
+  }
+  const int qraw = unit % args.nqblk;
+  const int qblk = args.reverse_q ? args.nqblk - 1 - qraw : qraw;
+  const int h = (unit / args.nqblk) % args.Hq;
+  const int b = unit / (args.nqblk * args.Hq);
   const int hk = h / args.group;
   const int q0 = qblk * 2 * kRowsPerTile;
 
@@ -208,6 +227,28 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     mbar_init(&s_free[0], kRowsPerTile);
     mbar_init(&s_free[1], kRowsPerTile);
     fence_mbar_init();
+    if (n_tiles > 0) {
+      // Q (and the rel tables) and the first K tile go out before the TMEM
+      // allocation and the CTA barrier, so their latency overlaps the setup
+      tma_prefetch_desc(&args.tq);
+      tma_prefetch_desc(&args.tk);
+      const int zq = b * args.Hq + h;
+      uint32_t qbytes = 2 * L::kQBytes;
+      if (KW > 0) qbytes += 2 * args.rel_n * 128;
+      mbar_expect_tx(q_full, qbytes);
+      for (int t = 0; t < 2; ++t)
+        for (int p = 0; p < L::kPanels; ++p)
+          tma_load_3d(sQ + t * L::kQBytes + p * kRowsPerTile * 128, &args.tq, q_full, p * 64,
+                      q0 + t * kRowsPerTile, zq);
+      if (KW > 0) {
+        // the rel tables borrow the last stage's K/V buffers until the projections are done
+        tma_load_3d(sK + (NS - 1) * L::kKVBytes, &args.trh, q_full, 0, 0, 0);
+        tma_load_3d(sV + (NS - 1) * L::kKVBytes, &args.trw, q_full, 0, 0, 0);
+      }
+      mbar_expect_tx(&k_full[0], L::kKVBytes);
+      for (int p = 0; p < L::kPanels; ++p)
+        tma_load_3d(sK + p * BN * 128, &args.tk, &k_full[0], p * 64, j_begin * BN, b * args.Hkv + hk);
+    }
   }
   if (warp == 9) {
     tmem_alloc(tslot, 512);
@@ -239,27 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_tiles > 0) {
-      tma_prefetch_desc(&args.tq);
-      tma_prefetch_desc(&args.tk);
       tma_prefetch_desc(&args.tv);
-      const int zq = b * args.Hq + h;
       const int zk = b * args.Hkv + hk;
-      uint32_t qbytes = 2 * L::kQBytes;
-      if (KW > 0) qbytes += 2 * args.rel_n * 128;
-      mbar_expect_tx(q_full, qbytes);
-      for (int t = 0; t < 2; ++t)
-        for (int p = 0; p < L::kPanels; ++p)
-          tma_load_3d(sQ + t * L::kQBytes + p * kRowsPerTile * 128, &args.tq, q_full, p * 64,
-                      q0 + t * kRowsPerTile, zq);
-      if (KW > 0) {
-        // the rel tables borrow the last stage's K/V buffers until the projections are done
-        tma_load_3d(sK + (NS - 1) * L::kKVBytes, &args.trh, q_full, 0, 0, 0);
-        tma_load_3d(sV + (NS - 1) * L::kKVBytes, &args.trw, q_full, 0, 0, 0);
-      }
       // K runs one tile ahead of V: a K stage frees as soon as both Q.K^T
       // products that read it are done, a V stage only after both P.V.
+      // Q, the rel tables and K tile 0 were issued during setup.
       bool ok = true;
-      int k_issued = 0, v_issued = 0;
+      int k_issued = 1, v_issued = 0;
       auto load_k = [&](int jj) {
         const int s = jj % NS, use = jj / NS;
         if (use > 0) ok = mbar_wait(&k_empty[s], (use - 1) & 1, abort_v, args.err);
@@ -282,9 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           tma_load_3d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, zk);
         v_issued = jj + 1;
       };
-      for (int jj = 0; jj < n_tiles && ok; ++jj) {
+      for (int jj = 1; jj < n_tiles && ok; ++jj) {
         load_k(jj);
-        if (ok && jj > 0) load_v(jj - 1);
+        if (ok) load_v(jj - 1);
       }
       if (ok) load_v(n_tiles - 1);
       if (!ok) {
@@ -450,7 +477,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         for (int w = 0; w < 2; ++w) {
           const int base_idx = w == 0 ? qh + kh_n - 1 : qw + KW - 1;
           const int nk = w == 0 ? kh_n : KW;
-          float* dst = w == 0 ? relh_s : relw_s;
 #pragma unroll
           for (int c0 = 0; c0 < 128; c0 += 32) {
             if (c0 < args.rel_n) {
@@ -460,26 +486,23 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int k = base_idx - (c0 + i);  // key-grid coordinate reached through table row c0+i
-                // [k][256] layout: consecutive rows hit consecutive banks whatever k is
-                if (k >= 0 && k < nk) dst[k * 256 + row] = __uint_as_float(r[i]) * kLog2e;
+                if (k >= 0 && k < nk) {
+                  const float val = __uint_as_float(r[i]) * kLog2e;
+                  if (w == 1 && kRwInSmem)
+                    // this row's slice, float4 groups XOR-swizzled by row: the
+                    // loop reads it as float4 without bank conflicts (and so
+                    // does this scatter when the query and key grids have equal width)
+                    relw_s[row * KW + ((((k >> 2) ^ (row & kRwSwz)) << 2) | (k & 3))] = val;
+                  else
+                    // [k][256]: consecutive rows hit consecutive banks whatever k is
+                    (w == 0 ? relh_s : relw_s)[k * 256 + row] = val;
+                }
               }
             }
           }
         }
       }
-      if constexpr (kRwInSmem) {
-        // Large key-grid width: the loop re-reads rel_w per tile as float4, so
-        // move this row's values into a row-major slice with float4 groups
-        // XOR-swizzled by row (conflict-free 128-bit reads), via registers.
-        float v[KW];
-#pragma unroll
-        for (int k = 0; k < KW; ++k) v[k] = relw_s[k * 256 + row];
-        named_bar_sync(1, 2 * kRowsPerTile);
-#pragma unroll
-        for (int k = 0; k < KW; k += 4)
-          *reinterpret_cast<float4*>(relw_s + row * KW + (((k >> 2) ^ (row & kRwSwz)) << 2)) =
-              make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-      }
+      // every thread reads back only what it wrote itself: no CTA barrier needed
       tc_fence_before();
       mbar_arrive(rel_read);
     }
@@ -646,6 +669,37 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         l_run *= alpha;
         m_run = m_new;
       }
+      // p = 2^(x + goff - m), packed to bf16 pairs in registers first, so that
+      // the wait for the previous P.V below comes after the exponentials.
+      // Some pairs take 2^y on the FMA pipe instead of the MUFU unit (only on
+      // tiles that hold no -inf: the polynomial path cannot return an exact 0).
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const bool emu = kEmuMask >= 0 && (MASK == TC_NONE) && (j0 + BN <= args.Tkv);
+      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int i = 0; i < BN / 2; ++i) {
+        const int c = 2 * i;
+        const float nmo = goff[c / GW] - m_use;
+        const uint64_t y2 = f2_add(x2[i], f2(nmo, nmo));
+        float p0, p1;
+        if (kEmuMask >= 0 && emu && (i & kEmuMask) == kEmuMask) {
+          f2_split(exp2_poly2(y2), p0, p1);
+        } else {
+          float lo, hi;
+          f2_split(y2, lo, hi);
+          p0 = ex2_approx(lo);
+          p1 = ex2_approx(hi);
+        }
+        sum2[i & 1] = f2_add(sum2[i & 1], f2(p0, p1));
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      {
+        float a0, a1, b0, b1;
+        f2_split(sum2[0], a0, a1);
+        f2_split(sum2[1], b0, b1);
+        l_run += (a0 + a1) + (b0 + b1);
+      }
       if constexpr (kPSep) {
         // O_t += P_t(j-1).V_{j-1} must be complete before O_t is rescaled or P_t is overwritten
         if (jj > 0) {
@@ -666,41 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           tmem_st32(o_addr + c0, r);
         }
       }
-
-      // p = 2^(x + goff - m), packed to bf16 pairs and written to P in TMEM.
-      // Some pairs take 2^y on the FMA pipe instead of the MUFU unit (only on
-      // tiles that hold no -inf: the polynomial path cannot return an exact 0).
-      const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const bool emu = kEmuMask >= 0 && (MASK == TC_NONE) && (j0 + BN <= args.Tkv);
-      uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t r8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = c0 + 2 * i;
-          const float nmo = goff[c / GW] - m_use;
-          const uint64_t y2 = f2_add(x2[c / 2], f2(nmo, nmo));
-          float p0, p1;
-          if (kEmuMask >= 0 && emu && ((c / 2) & kEmuMask) == kEmuMask) {
-            f2_split(exp2_poly2(y2), p0, p1);
-          } else {
-            float lo, hi;
-            f2_split(y2, lo, hi);
-            p0 = ex2_approx(lo);
-            p1 = ex2_approx(hi);
-          }
-          sum2[i & 1] = f2_add(sum2[i & 1], f2(p0, p1));
-          r8[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st8(p_addr + c0 / 2, r8);
-      }
-      {
-        float a0, a1, b0, b1;
-        f2_split(sum2[0], a0, a1);
-        f2_split(sum2[1], b0, b1);
-        l_run += (a0 + a1) + (b0 + b1);
-      }
+      for (int c0 = 0; c0 < BN / 2; c0 += 8) tmem_st8p(p_addr + c0, pk + c0);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -747,12 +768,15 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       }
     } else {
       // Split key range: publish this part (O unnormalised, running max m in
-      // log2 units, sum l); the last CTA of the block to arrive combines the
+      // log2 units, sum l); the last CTA of the unit to arrive combines the
       // parts, O = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k with M = max_k m_k.
-      const long long blk = zq * (gridDim.x / nsplit) + qblk;
-      float* wso = args.ws_o + ((blk * nsplit + sidx) * 256 + row) * D;
-      const bool have = n_tiles > 0 && ok && l_run > 0.f;
-      if (n_tiles > 0 && ok) {  // warp-uniform: the TMEM load is warp-collective
+      const long long part0 = (long long)(unit - args.n_full) * nsplit;
+      const bool live = n_tiles > 0 && ok;  // warp-uniform: the TMEM loads are warp-collective
+      const bool have = live && l_run > 0.f;
+      // partial O as [part][D/4][256 rows] float4: one store instruction of a
+      // warp writes 512 contiguous bytes
+      float4* wso = reinterpret_cast<float4*>(args.ws_o) + (part0 + sidx) * (D / 4) * 256 + row;
+      if (live) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t r[32];
@@ -761,37 +785,61 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           if (have) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
-              __stcg(reinterpret_cast<float4*>(wso + c0 + c),
+              __stcg(wso + ((c0 + c) / 4) * 256,
                      make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
                                  __uint_as_float(r[c + 3])));
           }
         }
       }
-      __stcg(args.ws_ml + (blk * nsplit + sidx) * 256 + row, make_float2(have ? m_run : -INFINITY, have ? l_run : 0.f));
-      __threadfence();
+      __stcg(args.ws_ml + (part0 + sidx) * 256 + row, make_float2(have ? m_run : -INFINITY, have ? l_run : 0.f));
+      // The barrier orders every thread's stores before thread 0's gpu-scope
+      // fence and ticket increment (fences are cumulative); the last arriver's
+      // fence after its increment acquires the other parts' stores.
       named_bar_sync(1, 2 * kRowsPerTile);
-      if (tid == 0) *reinterpret_cast<volatile int*>(abort_flag + 1) = atomicAdd(args.ws_cnt + blk, 1) == nsplit - 1;
+      if (tid == 0) {
+        fence_acq_rel_gpu();
+        const int last = atomicAdd(args.ws_cnt + (unit - args.n_full), 1) == nsplit - 1;
+        if (last) fence_acq_rel_gpu();
+        *reinterpret_cast<volatile int*>(abort_flag + 1) = last;
+      }
       named_bar_sync(1, 2 * kRowsPerTile);
       if (*reinterpret_cast<volatile int*>(abort_flag + 1)) {
-        __threadfence();
-        float M = -INFINITY;
-        for (int k = 0; k < nsplit; ++k) {
-          const float2 ml = __ldcg(args.ws_ml + (blk * nsplit + k) * 256 + row);
-          if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        // all (m, l) first (independent loads), then the weighted sum; this
+        // CTA's own part is still in TMEM
+        float2 ml[kMaxSplit];
+        float M = have ? m_run : -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kMaxSplit; ++k) {
+          ml[k] = make_float2(-INFINITY, 0.f);
+          if (k < nsplit && k != sidx) ml[k] = __ldcg(args.ws_ml + (part0 + k) * 256 + row);
+          if (ml[k].y > 0.f) M = fmaxf(M, ml[k].x);
         }
         float acc[D];
+        const float w_own = have ? ex2_approx(m_run - M) : 0.f;
+        float den = have ? w_own * l_run : 0.f;
 #pragma unroll
         for (int c = 0; c < D; ++c) acc[c] = 0.f;
-        float den = 0.f;
-        for (int k = 0; k < nsplit; ++k) {
-          const float2 ml = __ldcg(args.ws_ml + (blk * nsplit + k) * 256 + row);
-          if (ml.y > 0.f) {
-            const float w = ex2_approx(ml.x - M);
-            den = fmaf(w, ml.y, den);
-            const float* src = args.ws_o + ((blk * nsplit + k) * 256 + row) * D;
+        if (live) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(o_addr + c0, r);
+            tmem_wait_ld();
+            if (have) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) acc[c0 + c] = w_own * __uint_as_float(r[c]);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxSplit; ++k) {
+          if (ml[k].y > 0.f) {
+            const float w = ex2_approx(ml[k].x - M);
+            den = fmaf(w, ml[k].y, den);
+            const float4* src = reinterpret_cast<const float4*>(args.ws_o) + (part0 + k) * (D / 4) * 256 + row;
 #pragma unroll
             for (int c = 0; c < D; c += 4) {
-              const float4 o4 = __ldcg(reinterpret_cast<const float4*>(src + c));
+              const float4 o4 = __ldcg(src + (c / 4) * 256);
               acc[c] = fmaf(w, o4.x, acc[c]);
               acc[c + 1] = fmaf(w, o4.y, acc[c + 1]);
               acc[c + 2] = fmaf(w, o4.z, acc[c + 2]);
@@ -812,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           }
           if (args.lse) args.lse[zq * args.Tq + qi] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
         }
-        if (tid == 0) args.ws_cnt[blk] = 0;  // ready for the next launch
+        if (tid == 0) args.ws_cnt[unit - args.n_full] = 0;  // ready for the next launch
       }
     }
   }
@@ -909,6 +957,51 @@ int tc_check(const Params& p, sdpa_dtype_t dtype) {
   return SDPA_OK;
 }
 
+// Units (256-row query blocks of one (batch, head)) of a problem.
+long long nblk_of(const Params& p, int nqblk) { return (long long)nqblk * p.Hq * p.B; }
+// Key-tile width of the kernel instance the problem dispatches to.
+int BN_of(const Params& p) { return (p.use_rel && p.kw_n == 14) ? 112 : 128; }
+
+// Picks how many units run whole (first) and into how many parts each of the
+// rest is split, minimising the modelled time on nsm SMs with one CTA each.
+// A whole unit costs nt key tiles plus a fixed per-CTA cost (prologue,
+// epilogue); a part costs its share of the tiles, the fixed cost, and the
+// publish + merge of partial results.  Full waves of whole units go first and
+// the remainder is split finely enough to fill the last wave.  Causal /
+// sliding units differ in length and are not split.
+void tc_schedule(long long units, int nt, int nsm, bool ranged, bool rel, int* n_full, int* n_split) {
+  *n_full = (int)units;
+  *n_split = 1;
+  if (ranged || nt < 2 || units <= 0) return;
+  // fixed costs in key tiles (B200: ~2 us of prologue + epilogue per CTA, ~4.5 us with
+  // rel-pos projections; ~1.9 us per key tile of 2 x 128 rows at head_dim 64)
+  const double c0 = rel ? 4.0 : 2.0, cs = 2.0;
+  double best = (double)((units + nsm - 1) / nsm) * (nt + c0);
+  const long long full_waves = units / nsm;
+  for (long long fw = full_waves; fw >= 0 && fw >= full_waves - 1; --fw) {
+    const long long F = fw * nsm, R = units - F;
+    if (R <= 0) continue;
+    for (int sp = 2; sp <= kMaxSplit && sp <= nt; ++sp) {
+      const double waves_tail = (double)((R * sp + nsm - 1) / nsm);
+      const double cost = (double)fw * (nt + c0) + waves_tail * ((nt + sp - 1) / sp + c0 + cs);
+      if (cost < best - 1e-9) {
+        best = cost;
+        *n_full = (int)F;
+        *n_split = sp;
+      }
+    }
+  }
+#ifdef SDPA_TUNING
+  if (const char* e = getenv("SDPA_TC_SCHEDULE")) {  // "n_full,n_split" (tuning builds only)
+    int f = 0, sp = 1;
+    if (sscanf(e, "%d,%d", &f, &sp) == 2 && f >= 0 && f <= units && sp >= 1 && sp <= nt && sp <= kMaxSplit) {
+      *n_full = f;
+      *n_split = (f == units) ? 1 : sp;
+    }
+  }
+#endif
+}
+
 cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   TcArgs a;
   memset(&a, 0, sizeof(a));
@@ -942,36 +1035,24 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   a.err = p.err;
   const int nqblk = (p.Tq + 2 * kRowsPerTile - 1) / (2 * kRowsPerTile);
   const int mk = tc_mask_code(p);
-  // Fewer than two waves of query blocks: split each block's key range over
-  // several CTAs so the waves fill the SMs (parts merged in-kernel).
-  a.n_split = 1;
-  const long long nblk = (long long)nqblk * p.Hq * p.B;
-  const int nsm = num_sms();
-  const int nt = (p.Tkv + BN - 1) / BN;
-  if (mk != TC_RANGE && nblk < 2LL * nsm && nt >= 2) {
-    double best = 1e30;
-    for (int sp = 1; sp <= 8 && sp <= nt; ++sp) {
-      const double waves = (double)((nblk * sp + nsm - 1) / nsm);
-      // per-CTA fixed cost (prologue, partial write-out, merge) measured at
-      // about 16 key tiles' worth on B200
-      const double cost = waves * ((nt + sp - 1) / sp + 16.0);
-      if (cost < best - 1e-9) {
-        best = cost;
-        a.n_split = sp;
-      }
-    }
-  }
-  if (a.n_split > 1) {
-    const size_t nml = (size_t)nblk * a.n_split * 256 * sizeof(float2);
-    const size_t no = (size_t)nblk * a.n_split * 256 * p.d * sizeof(float);
+  tc_schedule(nblk_of(p, nqblk), (p.Tkv + BN_of(p) - 1) / BN_of(p), num_sms(), mk == TC_RANGE, p.use_rel != 0,
+              &a.n_full, &a.n_split);
+  a.nqblk = nqblk;
+  // causal: query blocks with the most key tiles first, so the short ones fill the tail
+  a.reverse_q = (mk == TC_RANGE && p.mask_kind == SDPA_MASK_CAUSAL) ? 1 : 0;
+  const long long units = nblk_of(p, nqblk);
+  const long long n_split_units = units - a.n_full;
+  if (n_split_units > 0) {
+    const size_t nml = (size_t)n_split_units * a.n_split * 256 * sizeof(float2);
+    const size_t no = (size_t)n_split_units * a.n_split * 256 * p.d * sizeof(float);
     void *cnt = nullptr, *data = nullptr;
-    if (workspace_get((size_t)nblk * sizeof(int), nml + no, &cnt, &data, stream) != SDPA_OK)
+    if (workspace_get((size_t)n_split_units * sizeof(int), nml + no, &cnt, &data, stream) != SDPA_OK)
       return cudaErrorMemoryAllocation;
     a.ws_cnt = static_cast<int*>(cnt);
     a.ws_ml = static_cast<float2*>(data);
     a.ws_o = reinterpret_cast<float*>(static_cast<char*>(data) + nml);
   }
-  dim3 grid((unsigned)(nqblk * a.n_split), (unsigned)p.Hq, (unsigned)p.B);
+  dim3 grid((unsigned)(a.n_full + n_split_units * a.n_split), 1u, 1u);
   if (!p.use_rel) {
     if (p.d == 64) return dispatch_mask<64, 128, 0, 3>(mk, a, grid, stream);
     return dispatch_mask<128, 128, 0, 2>(mk, a, grid, stream);
