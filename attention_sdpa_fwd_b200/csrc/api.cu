@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -277,10 +278,17 @@ extern "C" int sdpa_select_path(const void* q, const void* k, const void* v, voi
 namespace sdpa {
 namespace {
 
-// Device staging buffer of sdpa_fwd_host, one per device, grown on demand.
+// Slabs the host entry point pipelines a problem into.
+constexpr int kHostChunks = 6;
+
+// Device staging buffer of sdpa_fwd_host, one per device, grown on demand,
+// with the two copy streams and the events that order the pipeline.
 struct Staging {
   void* buf = nullptr;
   size_t cap = 0;
+  bool pipe_ready = false;
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t start = nullptr, landed[kHostChunks] = {}, computed[kHostChunks] = {};
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -332,30 +340,92 @@ extern "C" int sdpa_fwd_host(const void* q, const void* k, const void* v, void* 
     if (cudaMalloc(&st.buf, total) != cudaSuccess) return SDPA_ERR_CUDA;
     st.cap = total;
   }
+  if (!st.pipe_ready) {
+    if (cudaStreamCreateWithFlags(&st.up, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st.down, cudaStreamNonBlocking) != cudaSuccess)
+      return SDPA_ERR_CUDA;
+    for (int i = 0; i < kHostChunks; ++i)
+      if (cudaEventCreateWithFlags(&st.landed[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&st.computed[i], cudaEventDisableTiming) != cudaSuccess)
+        return SDPA_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&st.start, cudaEventDisableTiming) != cudaSuccess) return SDPA_ERR_CUDA;
+    st.pipe_ready = true;
+  }
   char* base = static_cast<char*>(st.buf);
-  auto h2d = [&](size_t off, const void* src, size_t n) {
-    return n == 0 || cudaMemcpyAsync(base + off, src, n, cudaMemcpyHostToDevice, stream) == cudaSuccess;
-  };
-  if (!h2d(oq, q, nq) || !h2d(ok, k, nk) || !h2d(ov, v, nk) || !h2d(orh, rel_pos_h, nrh) ||
-      !h2d(orw, rel_pos_w, nrw))
+  // Everything this call queues on the copy streams comes after the work
+  // already queued on the caller's stream.
+  if (cudaEventRecord(st.start, stream) != cudaSuccess || cudaStreamWaitEvent(st.up, st.start, 0) != cudaSuccess)
     return SDPA_ERR_CUDA;
+  auto h2d = [&](size_t off, const void* src, size_t n) {
+    return n == 0 || cudaMemcpyAsync(base + off, src, n, cudaMemcpyHostToDevice, st.up) == cudaSuccess;
+  };
+  if (!h2d(orh, rel_pos_h, nrh) || !h2d(orw, rel_pos_w, nrw)) return SDPA_ERR_CUDA;
   sdpa_mask_t dmask;
-  const void* mptr = mask_ptr;
   if (tensor_mask) {
     dmask = *static_cast<const sdpa_mask_t*>(mask_ptr);
     if (!h2d(om, dmask.data, nmask)) return SDPA_ERR_CUDA;
-    dmask.data = nmask ? base + om : nullptr;
-    mptr = &dmask;
   }
-  Problem dpr;
-  rc = build_problem(base + oq, Tkv ? base + ok : nullptr, Tkv ? base + ov : nullptr, base + oo, dtype, B,
-                     Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mptr, nrh ? base + orh : nullptr,
-                     nrw ? base + orw : nullptr, q_hw, k_hw, nullptr, &dpr);
-  if (rc != SDPA_OK) return rc;
-  rc = run(dpr, path, stream);
-  if (rc != SDPA_OK) return rc;
-  if (cudaMemcpyAsync(out, base + oo, nq, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return SDPA_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return SDPA_ERR_CUDA;
+
+  // Pipeline over slabs of (batch, head): slab i's inputs go up on one copy
+  // stream while slab i-1 computes on the caller's stream and slab i-2's
+  // output comes down on the other, so the copies overlap the kernels (and
+  // each other, on separate copy engines).  A slab is whole batches when
+  // there are at least kHostChunks of them, else a run of query heads of one
+  // batch that covers whole GQA groups.
+  const int group = Hq / Hkv;
+  struct Slab { int b0, nb, h0, nh; };
+  Slab slabs[kHostChunks];
+  int ns = 0;
+  if (B >= kHostChunks || Hq / group <= 1) {
+    const int per = (B + kHostChunks - 1) / kHostChunks;
+    for (int b0 = 0; b0 < B && ns < kHostChunks; b0 += per) slabs[ns++] = {b0, std::min(per, B - b0), 0, Hq};
+  } else {
+    const int groups = Hkv;                                   // kv heads per batch
+    const int per_b = std::max(1, kHostChunks / B);            // slabs per batch
+    const int gpc = (groups + per_b - 1) / per_b;              // kv groups per slab
+    for (int b = 0; b < B; ++b)
+      for (int g0 = 0; g0 < groups && ns < kHostChunks; g0 += gpc)
+        slabs[ns++] = {b, 1, g0 * group, std::min(gpc, groups - g0) * group};
+  }
+  const size_t qrow = (size_t)Tq * d * esz, krow = (size_t)Tkv * d * esz;  // bytes per (b, h)
+  const size_t mesz = mask_kind == SDPA_MASK_BOOL ? 1 : esz;
+  for (int i = 0; i < ns; ++i) {
+    const Slab& c = slabs[i];
+    const size_t zq0 = (size_t)c.b0 * Hq + c.h0, nzq = (size_t)c.nb * c.nh;        // (b, h) rows of q / out
+    const size_t zk0 = (size_t)c.b0 * Hkv + c.h0 / group, nzk = nzq / group;       // rows of k / v
+    const char* qh = static_cast<const char*>(q) + zq0 * qrow;
+    if (!h2d(oq + zq0 * qrow, qh, nzq * qrow)) return SDPA_ERR_CUDA;
+    if (Tkv > 0) {
+      if (!h2d(ok + zk0 * krow, static_cast<const char*>(k) + zk0 * krow, nzk * krow) ||
+          !h2d(ov + zk0 * krow, static_cast<const char*>(v) + zk0 * krow, nzk * krow))
+        return SDPA_ERR_CUDA;
+    }
+    if (cudaEventRecord(st.landed[i], st.up) != cudaSuccess || cudaStreamWaitEvent(stream, st.landed[i], 0) != cudaSuccess)
+      return SDPA_ERR_CUDA;
+    sdpa_mask_t cm;
+    const void* mptr = mask_ptr;
+    if (tensor_mask) {
+      cm = dmask;
+      cm.data = nmask ? base + om + ((long long)c.b0 * dmask.stride_b + (long long)c.h0 * dmask.stride_h) * mesz
+                      : nullptr;
+      mptr = &cm;
+    }
+    Problem dpr;
+    rc = build_problem(base + oq + zq0 * qrow, Tkv ? base + ok + zk0 * krow : nullptr,
+                       Tkv ? base + ov + zk0 * krow : nullptr, base + oo + zq0 * qrow, dtype, c.nb, c.nh,
+                       c.nh / group, Tq, Tkv, d, scale, mask_kind, mptr, nrh ? base + orh : nullptr,
+                       nrw ? base + orw : nullptr, q_hw, k_hw, nullptr, &dpr);
+    if (rc != SDPA_OK) return rc;
+    rc = run(dpr, path, stream);
+    if (rc != SDPA_OK) return rc;
+    if (cudaEventRecord(st.computed[i], stream) != cudaSuccess ||
+        cudaStreamWaitEvent(st.down, st.computed[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<char*>(out) + zq0 * qrow, base + oo + zq0 * qrow, nzq * qrow,
+                        cudaMemcpyDeviceToHost, st.down) != cudaSuccess)
+      return SDPA_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(st.down) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
+    return SDPA_ERR_CUDA;
   return SDPA_OK;
 }
 

@@ -219,3 +219,46 @@ def test_mixed_schedule(sp):
     assert_gates(out[:, :, rows].double().numpy(), ref.out, sp.dtype, sp.name)
     got = lse[:, :, rows].double().numpy()
     assert np.max(np.abs(got - ref.lse)) < 2e-3, "lse"
+
+
+HOST_CASES = [
+    # whole-batch slabs (B >= 6), per-head float mask with -inf entries
+    S_("host_batches_float_mask", BF16, 7, 4, 2, 200, 150, 64, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=4, seed=60),
+    # head slabs covering whole GQA groups (group of 4)
+    S_("host_gqa_head_slabs", BF16, 1, 8, 2, 300, 260, 128, mask_kind=W.MASK_CAUSAL, seed=61),
+    # rel-pos, several slabs per batch
+    S_("host_relpos_slabs", BF16, 2, 6, 6, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5, seed=62),
+]
+
+
+@pytest.mark.parametrize("sp", HOST_CASES, ids=[c.name for c in HOST_CASES])
+def test_host_entry_point_slabs(sp):
+    """sdpa_fwd_host pipelines the problem over (batch, head) slabs; the bytes
+    must equal the device entry point's, and the values the oracle's."""
+    import ctypes
+    import attention_sdpa_fwd_b200 as S
+    wl = W.make(sp)
+    dev_out, _ = gpu_run(wl)
+    pin = lambda x: None if x is None else x.contiguous().pin_memory()
+    qh, kh, vh, mh = pin(wl.q), pin(wl.k), pin(wl.v), pin(wl.mask)
+    rh = wl.rel_pos_h.contiguous() if wl.rel_pos_h is not None else None
+    rw = wl.rel_pos_w.contiguous() if wl.rel_pos_w is not None else None
+    out = torch.empty_like(qh).pin_memory()
+    m = None
+    if sp.mask_kind != W.MASK_NONE:
+        m = S.sdpa_mask_t(offset=sp.offset, window=sp.window, data=None, stride_b=0, stride_h=0, stride_q=0)
+        if mh is not None:
+            m.data = mh.data_ptr()
+            m.stride_b = 0 if mh.shape[0] == 1 else mh.stride(0)
+            m.stride_h = 0 if mh.shape[1] == 1 else mh.stride(1)
+            m.stride_q = mh.stride(2)
+    rc = S.sdpa_fwd_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), out.data_ptr(), S.SDPA_BF16,
+                         sp.B, sp.Hq, sp.Hkv, sp.Tq, sp.Tkv, sp.d, sp.scale, sp.mask_kind,
+                         ctypes.byref(m) if m is not None else None,
+                         rh.data_ptr() if rh is not None else None, rw.data_ptr() if rw is not None else None,
+                         sp.q_hw, sp.k_hw, 0, torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    assert torch.equal(out, dev_out)
+    ref = oracle_ref(wl)
+    assert_gates(out.double().numpy(), ref.out, sp.dtype, sp.name)
