@@ -26,6 +26,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace sdpa {
 namespace {
@@ -65,9 +66,9 @@ __device__ __forceinline__ float mask_term(const Params& p, long long mrow, long
 constexpr int kRowsPerCta = 128;
 constexpr int kKeyChunk = 128;
 
-__global__ void __launch_bounds__(kRowsPerCta) small_d_kernel(Params p) {
-  __shared__ float sk[kKeyChunk][D16];
-  __shared__ float sv[kKeyChunk][D16];
+__global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p) {
+  __shared__ float4 sk[kKeyChunk][D16 / 4];  // every thread reads the same key: broadcast
+  __shared__ float4 sv[kKeyChunk][D16 / 4];
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.group;
   const long long i = (long long)blockIdx.x * kRowsPerCta + threadIdx.x;
@@ -108,31 +109,57 @@ __global__ void __launch_bounds__(kRowsPerCta) small_d_kernel(Params p) {
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * D16)), f);
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * D16) + 1), f + 8);
 #pragma unroll
-      for (int c = 0; c < D16; ++c) sk[threadIdx.x][c] = f[c];
+      for (int c = 0; c < D16; c += 4) sk[threadIdx.x][c / 4] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * D16)), f);
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * D16) + 1), f + 8);
 #pragma unroll
-      for (int c = 0; c < D16; ++c) sv[threadIdx.x][c] = f[c];
+      for (int c = 0; c < D16; c += 4) sv[threadIdx.x][c / 4] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
     }
     __syncthreads();
     if (!valid) continue;
-    for (int t = 0; t < n; ++t) {
-      float s = 0.f;
+    // eight keys at a time: scores, their max, one rescale, then the sums
+    for (int t0 = 0; t0 < n; t0 += 8) {
+      float sc[8];
+      float cmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < D16; ++c) s = fmaf(q[c], sk[t][c], s);
-      if (elementwise) s += mask_term(p, mrow, i, j0 + t);
-      if (s == -INFINITY) continue;
-      if (s > m) {
-        const float corr = exp2f(m - s);  // 0 when m == -inf
+      for (int u = 0; u < 8; ++u) {
+        const int t = t0 + u;
+        float x = -INFINITY;
+        if (t < n) {
+          x = 0.f;
+#pragma unroll
+          for (int c = 0; c < D16; c += 4) {
+            const float4 k4 = sk[t][c / 4];
+            x = fmaf(q[c], k4.x, fmaf(q[c + 1], k4.y, fmaf(q[c + 2], k4.z, fmaf(q[c + 3], k4.w, x))));
+          }
+          if (elementwise) x += mask_term(p, mrow, i, j0 + t);
+        }
+        sc[u] = x;
+        cmax = fmaxf(cmax, x);
+      }
+      if (cmax == -INFINITY) continue;
+      if (cmax > m) {
+        const float corr = sm100::ex2_approx(m - cmax);  // 0 when m == -inf
         l *= corr;
 #pragma unroll
         for (int c = 0; c < D16; ++c) acc[c] *= corr;
-        m = s;
+        m = cmax;
       }
-      const float pj = exp2f(s - m);
-      l += pj;
 #pragma unroll
-      for (int c = 0; c < D16; ++c) acc[c] = fmaf(pj, sv[t][c], acc[c]);
+      for (int u = 0; u < 8; ++u) {
+        const float pj = sm100::ex2_approx(sc[u] - m);  // 0 for -inf
+        l += pj;
+        if (t0 + u < n) {
+#pragma unroll
+          for (int c = 0; c < D16; c += 4) {
+            const float4 v4 = sv[t0 + u][c / 4];
+            acc[c] = fmaf(pj, v4.x, acc[c]);
+            acc[c + 1] = fmaf(pj, v4.y, acc[c + 1]);
+            acc[c + 2] = fmaf(pj, v4.z, acc[c + 2]);
+            acc[c + 3] = fmaf(pj, v4.w, acc[c + 3]);
+          }
+        }
+      }
     }
   }
   if (!valid) return;
@@ -165,10 +192,12 @@ struct SplitArgs {
   int* ws_cnt;     // [B*Hq] tickets, zero between launches
 };
 
-__global__ void __launch_bounds__(kSplitThreads) split_kv_kernel(SplitArgs a) {
+__global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a) {
   const Params& p = a.p;
-  __shared__ float sk[kSplitChunk][D16 + 1];
-  __shared__ float sv[kSplitChunk][D16 + 1];
+  // key t's row as four float4 at [t][f ^ ((t >> 1) & 3)]: eight consecutive
+  // lanes reading the same f of consecutive keys hit all 32 banks once
+  __shared__ float4 sk[kSplitChunk][D16 / 4];
+  __shared__ float4 sv[kSplitChunk][D16 / 4];
   __shared__ int s_last;
   const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.group;
@@ -182,11 +211,11 @@ __global__ void __launch_bounds__(kSplitThreads) split_kv_kernel(SplitArgs a) {
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * D16)), f);
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * D16) + 1), f + 8);
 #pragma unroll
-    for (int c = 0; c < D16; ++c) sk[t][c] = f[c];
+    for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * D16)), f);
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * D16) + 1), f + 8);
 #pragma unroll
-    for (int c = 0; c < D16; ++c) sv[t][c] = f[c];
+    for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,23 +229,42 @@ __global__ void __launch_bounds__(kSplitThreads) split_kv_kernel(SplitArgs a) {
     float m = -INFINITY, l = 0.f, acc[D16];
 #pragma unroll
     for (int c = 0; c < D16; ++c) acc[c] = 0.f;
-    for (int t = lane; t < n; t += 32) {
-      float s = 0.f;
+    // this lane's keys (lane, lane + 32, ... : at most kSplitChunk / 32 of
+    // them): scores, their max, then the sums
+    float sc[kSplitChunk / 32];
 #pragma unroll
-      for (int c = 0; c < D16; ++c) s = fmaf(q[c], sk[t][c], s);
-      s = s * sl + mask_term(p, mrow, i, j0 + t);
-      if (s == -INFINITY) continue;
-      if (s > m) {
-        const float corr = exp2f(m - s);
-        l *= corr;
+    for (int u = 0; u < kSplitChunk / 32; ++u) {
+      const int t = lane + 32 * u;
+      float x = -INFINITY;
+      if (t < n) {
+        x = 0.f;
 #pragma unroll
-        for (int c = 0; c < D16; ++c) acc[c] *= corr;
-        m = s;
+        for (int c = 0; c < D16; c += 4) {
+          const float4 k4 = sk[t][(c / 4) ^ ((t >> 1) & 3)];
+          x = fmaf(q[c], k4.x, fmaf(q[c + 1], k4.y, fmaf(q[c + 2], k4.z, fmaf(q[c + 3], k4.w, x))));
+        }
+        x = x * sl + mask_term(p, mrow, i, j0 + t);
       }
-      const float pj = exp2f(s - m);
-      l += pj;
+      sc[u] = x;
+      m = fmaxf(m, x);
+    }
+    if (m != -INFINITY) {
 #pragma unroll
-      for (int c = 0; c < D16; ++c) acc[c] = fmaf(pj, sv[t][c], acc[c]);
+      for (int u = 0; u < kSplitChunk / 32; ++u) {
+        const int t = lane + 32 * u;
+        const float pj = sm100::ex2_approx(sc[u] - m);  // 0 for -inf
+        l += pj;
+        if (t < n) {
+#pragma unroll
+          for (int c = 0; c < D16; c += 4) {
+            const float4 v4 = sv[t][(c / 4) ^ ((t >> 1) & 3)];
+            acc[c] = fmaf(pj, v4.x, acc[c]);
+            acc[c + 1] = fmaf(pj, v4.y, acc[c + 1]);
+            acc[c + 2] = fmaf(pj, v4.z, acc[c + 2]);
+            acc[c + 3] = fmaf(pj, v4.w, acc[c + 3]);
+          }
+        }
+      }
     }
     // combine the 32 lanes
     float M = m;
@@ -226,47 +274,79 @@ __global__ void __launch_bounds__(kSplitThreads) split_kv_kernel(SplitArgs a) {
     l *= w;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    // sum the 16 columns over the 32 lanes as a butterfly reduce-scatter:
+    // at each step a lane keeps half of its columns and adds its partner's
+    // half (8 + 4 + 2 + 1 + 1 shuffles instead of 16 x 5); lane pair
+    // (2k, 2k+1) ends with column col = bits 4..1 of the lane
 #pragma unroll
-    for (int c = 0; c < D16; ++c) {
-      float x = acc[c] * w;
+    for (int c = 0; c < D16; ++c) acc[c] *= w;
+    const long long slot = (zq * a.nsplit + part) * p.Tq + i;
+    float r8[8], r4[4], r2[2], r1;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-      acc[c] = x;
+    for (int k = 0; k < 8; ++k) {
+      const bool hi = lane & 16;
+      r8[k] = (hi ? acc[k + 8] : acc[k]) + __shfl_xor_sync(0xffffffffu, hi ? acc[k] : acc[k + 8], 16);
     }
-    if (lane == 0) {
-      const long long slot = (zq * a.nsplit + part) * p.Tq + i;
-      float4* dst = reinterpret_cast<float4*>(a.ws_o + slot * D16);
 #pragma unroll
-      for (int c = 0; c < D16; c += 4) __stcg(dst + c / 4, make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
-      __stcg(a.ws_ml + slot, make_float2(M, l));
+    for (int k = 0; k < 4; ++k) {
+      const bool hi = lane & 8;
+      r4[k] = (hi ? r8[k + 4] : r8[k]) + __shfl_xor_sync(0xffffffffu, hi ? r8[k] : r8[k + 4], 8);
     }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const bool hi = lane & 4;
+      r2[k] = (hi ? r4[k + 2] : r4[k]) + __shfl_xor_sync(0xffffffffu, hi ? r4[k] : r4[k + 2], 4);
+    }
+    {
+      const bool hi = lane & 2;
+      r1 = (hi ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, hi ? r2[0] : r2[1], 2);
+    }
+    r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+    if ((lane & 1) == 0) {
+      const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+      __stcg(a.ws_o + slot * D16 + col, r1);
+    }
+    if (lane == 0) __stcg(a.ws_ml + slot, make_float2(M, l));
   }
-  // the last part of this (batch, head) to finish merges all parts
-  __threadfence();
+  // the last part of this (batch, head) to finish merges all parts.  The CTA
+  // barrier orders every thread's stores before thread 0's gpu-scope fence
+  // and ticket increment (fences are cumulative); the last arriver's fence
+  // after its increment acquires the other parts' stores.
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(a.ws_cnt + zq, 1) == a.nsplit - 1;
+  if (threadIdx.x == 0) {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    s_last = atomicAdd(a.ws_cnt + zq, 1) == a.nsplit - 1;
+    if (s_last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
+  const long long base = zq * a.nsplit;  // first part slot of this (batch, head)
   for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
-    // lanes 0..15 own one output column each
+    // M = max over parts (one part per lane), then lanes (c, half) = (lane & 15,
+    // lane >> 4) sum column c over every other part: independent loads, no
+    // chain of round trips through the parts
     float M = -INFINITY;
     for (int k = lane; k < a.nsplit; k += 32) {
-      const float2 ml = __ldcg(a.ws_ml + (zq * a.nsplit + k) * p.Tq + i);
+      const float2 ml = __ldcg(a.ws_ml + (base + k) * p.Tq + i);
       if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const int c = lane & 15;
     float den = 0.f, num = 0.f;
-    for (int k = 0; k < a.nsplit; ++k) {
-      const long long slot = (zq * a.nsplit + k) * p.Tq + i;
+#pragma unroll 4
+    for (int k = lane >> 4; k < a.nsplit; k += 2) {
+      const long long slot = (base + k) * p.Tq + i;
       const float2 ml = __ldcg(a.ws_ml + slot);
+      const float o = __ldcg(a.ws_o + slot * D16 + c);
       if (ml.y > 0.f) {
         const float w = exp2f(ml.x - M);
         den = fmaf(w, ml.y, den);
-        if (lane < D16) num = fmaf(w, __ldcg(a.ws_o + slot * D16 + lane), num);
+        num = fmaf(w, o, num);
       }
     }
+    den += __shfl_xor_sync(0xffffffffu, den, 16);
+    num += __shfl_xor_sync(0xffffffffu, num, 16);
     const float val = den > 0.f ? num / den : 0.f;
     const float nb = __shfl_down_sync(0xffffffffu, val, 1);
     if (lane < D16 && (lane & 1) == 0) {
