@@ -26,8 +26,8 @@ STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
           -6: "SDPA_ERR_CAPACITY"}
 
 # Every symbol include/sdpa.h declares.
-EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_select_path", "sdpa_fwd_host", "sdpa_fwd_split_kv_static",
-           "sdpa_last_device_error", "sdpa_strerror", "sdpa_version")
+EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_select_path", "sdpa_fwd_host",
+           "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_strerror", "sdpa_version")
 
 
 class SdpaError(RuntimeError):
@@ -39,6 +39,10 @@ class SdpaError(RuntimeError):
 class sdpa_mask_t(ctypes.Structure):
     _fields_ = [("offset", ctypes.c_int64), ("window", ctypes.c_int64), ("data", ctypes.c_void_p),
                 ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64), ("stride_q", ctypes.c_int64)]
+
+
+class sdpa_strides_t(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("t", ctypes.c_int64)]
 
 
 _lib = None
@@ -57,12 +61,13 @@ def lib():
         L.sdpa_fwd.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
         L.sdpa_fwd_ex.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
         L.sdpa_fwd_host.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+        L.sdpa_fwd_strided.argtypes = [_vp] * 8 + [_i32] * 7 + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
         L.sdpa_select_path.argtypes = _COMMON + [_i32, _vp, _vp, _vp, _vp, _vp]
         L.sdpa_fwd_split_kv_static.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp]
         L.sdpa_last_device_error.argtypes = [_vp]
         L.sdpa_strerror.argtypes = [_i32]
         L.sdpa_strerror.restype = ctypes.c_char_p
-        for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_host", "sdpa_select_path",
+        for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_fwd_host", "sdpa_select_path",
                      "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_version"):
             getattr(L, name).restype = _i32
         _lib = L
@@ -86,6 +91,14 @@ def sdpa_fwd_ex(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, m
                 rel_pos_h, rel_pos_w, q_hw, k_hw, lse, path, stream) -> int:
     return lib().sdpa_fwd_ex(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
                              rel_pos_h, rel_pos_w, _hw(q_hw), _hw(k_hw), lse, path, stream)
+
+
+def sdpa_fwd_strided(q, q_strides, k, k_strides, v, v_strides, out, out_strides, dtype, B, Hq, Hkv, Tq, Tkv,
+                     d, scale, mask_kind, mask_ptr, rel_pos_h, rel_pos_w, q_hw, k_hw, lse, path, stream) -> int:
+    st = lambda x: None if x is None else ctypes.byref(sdpa_strides_t(*(int(y) for y in x)))
+    return lib().sdpa_fwd_strided(q, st(q_strides), k, st(k_strides), v, st(v_strides), out, st(out_strides),
+                                  dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr, rel_pos_h, rel_pos_w,
+                                  _hw(q_hw), _hw(k_hw), lse, path, stream)
 
 
 def sdpa_fwd_host(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
@@ -156,29 +169,44 @@ def sdpa(q, k, v, scale: Optional[float] = None, *, mask_kind: int = MASK_NONE, 
          window: int = 0, mask=None, rel_pos_h=None, rel_pos_w=None,
          q_hw: Optional[Sequence[int]] = None, k_hw: Optional[Sequence[int]] = None,
          out=None, lse=None, path: str = "auto", stream=None):
-    """softmax(q.k^T*scale + bias).v on CUDA tensors in bhsd layout.
+    """softmax(q.k^T*scale + bias).v on CUDA tensors indexed [B, H, T, d].
 
-    q [B,Hq,Tq,d], k/v [B,Hkv,Tkv,d], contiguous, float32 or bfloat16.
-    ``scale`` defaults to 1/sqrt(d) (Axon PR, :scale option).  Returns ``out``."""
+    q [B,Hq,Tq,d], k/v [B,Hkv,Tkv,d], float32 or bfloat16, with a contiguous
+    last axis and any batch / head / token strides: a "bshd" tensor [B,T,H,d]
+    passed as x.transpose(1, 2) is used in place (sdpa_fwd_strided), dense
+    bhsd tensors go through sdpa_fwd_ex.  ``out`` (allocated bhsd when None)
+    may be strided the same way.  ``scale`` defaults to 1/sqrt(d) (Axon PR,
+    :scale option).  Returns ``out``."""
     import torch
     for t in (q, k, v):
         if not t.is_cuda:
             raise ValueError("sdpa runs on CUDA tensors only (no CPU fallback)")
-        if not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous (bhsd)")
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError("q, k, v must be 4-D [B, H, T, d] with a contiguous last axis")
     B, Hq, Tq, d = q.shape
     Hkv, Tkv = k.shape[1], k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, Hq, Tq, d), device=q.device, dtype=q.dtype)
+    elif out.dim() != 4 or out.stride(3) != 1:
+        raise ValueError("out must be 4-D with a contiguous last axis")
     m = make_mask(mask_kind, offset=offset, window=window, tensor=mask)
     st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    mp = ctypes.byref(m) if m is not None else None
     with torch.cuda.device(q.device):
-        rc = sdpa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, Hq, Hkv, Tq, Tkv, d,
-                         float(scale), mask_kind, ctypes.byref(m) if m is not None else None,
-                         _ptr(rel_pos_h), _ptr(rel_pos_w), q_hw, k_hw, _ptr(lse), PATHS[path],
-                         st.cuda_stream)
+        if all(t.is_contiguous() for t in (q, k, v, out)):
+            rc = sdpa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, Hq, Hkv, Tq, Tkv, d,
+                             float(scale), mask_kind, mp, _ptr(rel_pos_h), _ptr(rel_pos_w), q_hw, k_hw,
+                             _ptr(lse), PATHS[path], st.cuda_stream)
+            what = "sdpa_fwd_ex"
+        else:
+            s3 = lambda t: (t.stride(0), t.stride(1), t.stride(2))
+            rc = sdpa_fwd_strided(_ptr(q), s3(q), _ptr(k), s3(k), _ptr(v), s3(v), _ptr(out), s3(out),
+                                  _dtype_code(q), B, Hq, Hkv, Tq, Tkv, d, float(scale), mask_kind, mp,
+                                  _ptr(rel_pos_h), _ptr(rel_pos_w), q_hw, k_hw, _ptr(lse), PATHS[path],
+                                  st.cuda_stream)
+            what = "sdpa_fwd_strided"
     if rc != 0:
-        raise SdpaError(rc, "sdpa_fwd_ex")
+        raise SdpaError(rc, what)
     return out

@@ -69,7 +69,8 @@ struct Problem {
 int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype, int B,
                   int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
                   const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
-                  const int* q_hw, const int* k_hw, float* lse, Problem* pr) {
+                  const int* q_hw, const int* k_hw, float* lse, Problem* pr,
+                  const sdpa_strides_t* const* strides = nullptr) {
   memset(pr, 0, sizeof(*pr));
   if (dtype != SDPA_F32 && dtype != SDPA_BF16) return SDPA_ERR_INVALID_ARG;
   if (B < 0 || Hq < 1 || Hkv < 1 || Tq < 0 || Tkv < 0) return SDPA_ERR_INVALID_ARG;
@@ -88,6 +89,26 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
   pr->empty_out = rows == 0;
   pr->dtype = dtype;
   pr->esz = esz;
+  // strides: dense bhsd unless given
+  {
+    const long long dq[3] = {(long long)Hq * Tq * d, (long long)Tq * d, d};
+    const long long dk[3] = {(long long)Hkv * Tkv * d, (long long)Tkv * d, d};
+    long long* dst[4][3] = {{&p.sqb, &p.sqh, &p.sqt}, {&p.skb, &p.skh, &p.skt},
+                            {&p.svb, &p.svh, &p.svt}, {&p.sob, &p.soh, &p.sot}};
+    for (int a = 0; a < 4; ++a) {
+      const long long* def = (a == 1 || a == 2) ? dk : dq;
+      const sdpa_strides_t* st = strides ? strides[a] : nullptr;
+      if (st == nullptr) {
+        for (int x = 0; x < 3; ++x) *dst[a][x] = def[x];
+      } else {
+        const long long given[3] = {st->b, st->h, st->t};
+        for (int x = 0; x < 3; ++x) {
+          if (given[x] < 1 || given[x] > (1LL << 40)) return SDPA_ERR_INVALID_ARG;
+          *dst[a][x] = given[x];
+        }
+      }
+    }
+  }
 
   const sdpa_mask_t* m = static_cast<const sdpa_mask_t*>(mask_ptr);
   if (mask_kind == SDPA_MASK_CAUSAL) {
@@ -127,14 +148,21 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
     if (!aligned(q, esz) || !aligned(out, esz) || (k && !aligned(k, esz)) || (v && !aligned(v, esz)))
       return SDPA_ERR_MISALIGNED;
     if (lse && !aligned(lse, 4)) return SDPA_ERR_MISALIGNED;
-    const size_t nq = (size_t)rows * d * esz;
-    const size_t nk = (size_t)B * Hkv * Tkv * d * esz;
-    if (overlaps(out, nq, q, nq) || overlaps(out, nq, k, nk) || overlaps(out, nq, v, nk))
+    // address span of each tensor: last element + 1, in bytes
+    auto span = [&](long long sb, long long sh, long long st, int H, int T) -> size_t {
+      if (B == 0 || T == 0) return 0;
+      return (size_t)((B - 1) * sb + (long long)(H - 1) * sh + (long long)(T - 1) * st + d) * esz;
+    };
+    const size_t nq = span(p.sqb, p.sqh, p.sqt, Hq, Tq), no = span(p.sob, p.soh, p.sot, Hq, Tq);
+    const size_t nk = span(p.skb, p.skh, p.skt, Hkv, Tkv), nv = span(p.svb, p.svh, p.svt, Hkv, Tkv);
+    if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
       return SDPA_ERR_INVALID_ARG;
-    if (lse && (overlaps(lse, (size_t)rows * 4, out, nq) || overlaps(lse, (size_t)rows * 4, q, nq)))
+    if (lse && (overlaps(lse, (size_t)rows * 4, out, no) || overlaps(lse, (size_t)rows * 4, q, nq)))
       return SDPA_ERR_INVALID_ARG;
   }
-  p.k_vec16 = (k != nullptr && aligned(k, 16)) ? 1 : 0;
+  p.k_vec16 = (k != nullptr && aligned(k, 16) && (p.skb * (long long)esz) % 16 == 0 &&
+               (p.skh * (long long)esz) % 16 == 0 && (p.skt * (long long)esz) % 16 == 0)
+                  ? 1 : 0;
   return SDPA_OK;
 }
 
@@ -251,6 +279,21 @@ extern "C" int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* ou
   Problem pr;
   int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
                          rel_pos_h, rel_pos_w, q_hw, k_hw, lse, &pr);
+  if (rc != SDPA_OK) return rc;
+  return run(pr, path, stream);
+}
+
+extern "C" int sdpa_fwd_strided(const void* q, const sdpa_strides_t* q_strides, const void* k,
+                                const sdpa_strides_t* k_strides, const void* v, const sdpa_strides_t* v_strides,
+                                void* out, const sdpa_strides_t* out_strides, sdpa_dtype_t dtype, int B, int Hq,
+                                int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind, const void* mask_ptr,
+                                const void* rel_pos_h, const void* rel_pos_w, const int* q_hw, const int* k_hw,
+                                float* lse, int path, cudaStream_t stream) {
+  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_SPLIT_KV) return SDPA_ERR_INVALID_ARG;
+  const sdpa_strides_t* st[4] = {q_strides, k_strides, v_strides, out_strides};
+  Problem pr;
+  int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
+                         rel_pos_h, rel_pos_w, q_hw, k_hw, lse, &pr, st);
   if (rc != SDPA_OK) return rc;
   return run(pr, path, stream);
 }

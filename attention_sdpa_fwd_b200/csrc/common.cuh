@@ -28,8 +28,31 @@ struct Params {
   int use_rel;
   int qh_n, qw_n, kh_n, kw_n;  // query / key patch grids (height, width)
   int* err;          // device error word (bounded waits report here)
-  int k_vec16;       // k's base is 16-byte aligned (vector loads allowed)
+  int k_vec16;       // k's rows are 16-byte aligned (vector loads allowed)
+  // element strides of the batch, head and token axes (head_dim contiguous)
+  long long sqb, sqh, sqt, skb, skh, skt, svb, svh, svt, sob, soh, sot;
 };
+
+// Element offsets of row t of (batch b, head h) in q / k / v / out.
+__host__ __device__ __forceinline__ long long q_off(const Params& p, long long b, long long h, long long t) {
+  return b * p.sqb + h * p.sqh + t * p.sqt;
+}
+__host__ __device__ __forceinline__ long long k_off(const Params& p, long long b, long long h, long long t) {
+  return b * p.skb + h * p.skh + t * p.skt;
+}
+__host__ __device__ __forceinline__ long long v_off(const Params& p, long long b, long long h, long long t) {
+  return b * p.svb + h * p.svh + t * p.svt;
+}
+__host__ __device__ __forceinline__ long long o_off(const Params& p, long long b, long long h, long long t) {
+  return b * p.sob + h * p.soh + t * p.sot;
+}
+// Every stride of q, k, v and out is a multiple of n elements.
+__host__ __device__ __forceinline__ bool strides_multiple_of(const Params& p, long long n) {
+  const long long s[12] = {p.sqb, p.sqh, p.sqt, p.skb, p.skh, p.skt, p.svb, p.svh, p.svt, p.sob, p.soh, p.sot};
+  for (int i = 0; i < 12; ++i)
+    if (s[i] % n != 0) return false;
+  return true;
+}
 
 enum ErrBits { ERR_WAIT_TIMEOUT = 1 };
 

@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
   float* relh = qs + D;
   float* relw = relh + p.kh_n;
 
-  const T* qrow = static_cast<const T*>(p.q) + (((long long)b * p.Hq + h) * p.Tq + i) * D;
+  const T* qrow = static_cast<const T*>(p.q) + q_off(p, b, h, i);
   for (int c = lane; c < D; c += 32) qs[c] = to_f32(qrow[c]);
   __syncwarp();
 
@@ -81,8 +81,8 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
   const bool owns_cols = (D >= 32) || (lane < D);
   const int col0 = D >= 32 ? lane * CPL : lane;
 
-  const T* kb = static_cast<const T*>(p.k) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D;
-  const T* vb = static_cast<const T*>(p.v) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D;
+  const T* kb = static_cast<const T*>(p.k) + k_off(p, b, hk, 0);
+  const T* vb = static_cast<const T*>(p.v) + v_off(p, b, hk, 0);
   const long long mrow = (long long)b * p.msb + (long long)h * p.msh + i * p.msq;
 
   float m = -INFINITY, l = 0.f;
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     const long long j = j0 + lane;
     float s = -INFINITY;
     if (j < hi) {
-      s = p.scale * (p.k_vec16 ? dot_row<T, D>(qs, kb + j * D) : dot_any<T>(qs, kb + j * D, D));
+      s = p.scale * (p.k_vec16 ? dot_row<T, D>(qs, kb + j * p.skt) : dot_any<T>(qs, kb + j * p.skt, D));
       if (p.use_rel) s += relh[j / p.kw_n] + relw[j % p.kw_n];
       if (p.mask_kind == SDPA_MASK_ADD_FLOAT) {
         s += to_f32(static_cast<const T*>(p.mask)[mrow + j]);
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     for (int t = 0; t < nk; ++t) {
       const float pt = __shfl_sync(0xffffffffu, pj, t);
       if (owns_cols) {
-        const T* vr = vb + (j0 + t) * D + col0;
+        const T* vr = vb + (j0 + t) * p.svt + col0;
 #pragma unroll
         for (int c = 0; c < CPL; ++c) acc[c] = fmaf(pt, to_f32(vr[c]), acc[c]);
       }
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
   }
 
   const float inv = l > 0.f ? 1.f / l : 0.f;
-  T* orow = static_cast<T*>(p.out) + (((long long)b * p.Hq + h) * p.Tq + i) * D;
+  T* orow = static_cast<T*>(p.out) + o_off(p, b, h, i);
   if (owns_cols) {
 #pragma unroll
     for (int c = 0; c < CPL; ++c) orow[col0 + c] = from_f32<T>(acc[c] * inv);

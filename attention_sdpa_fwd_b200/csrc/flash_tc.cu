@@ -72,6 +72,7 @@ enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3 };
 struct TcArgs {
   CUtensorMap tq, tk, tv, trh, trw;
   void* out;
+  long long sob, soh, sot;  // element strides of out (batch, head, token)
   float* lse;
   const void* mask;
   long long msb, msh, msq;
@@ -232,14 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       // allocation and the CTA barrier, so their latency overlaps the setup
       tma_prefetch_desc(&args.tq);
       tma_prefetch_desc(&args.tk);
-      const int zq = b * args.Hq + h;
       uint32_t qbytes = 2 * L::kQBytes;
       if (KW > 0) qbytes += 2 * args.rel_n * 128;
       mbar_expect_tx(q_full, qbytes);
       for (int t = 0; t < 2; ++t)
         for (int p = 0; p < L::kPanels; ++p)
-          tma_load_3d(sQ + t * L::kQBytes + p * kRowsPerTile * 128, &args.tq, q_full, p * 64,
-                      q0 + t * kRowsPerTile, zq);
+          tma_load_4d(sQ + t * L::kQBytes + p * kRowsPerTile * 128, &args.tq, q_full, p * 64,
+                      q0 + t * kRowsPerTile, h, b);
       if (KW > 0) {
         // the rel tables borrow the last stage's K/V buffers until the projections are done
         tma_load_3d(sK + (NS - 1) * L::kKVBytes, &args.trh, q_full, 0, 0, 0);
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       }
       mbar_expect_tx(&k_full[0], L::kKVBytes);
       for (int p = 0; p < L::kPanels; ++p)
-        tma_load_3d(sK + p * BN * 128, &args.tk, &k_full[0], p * 64, j_begin * BN, b * args.Hkv + hk);
+        tma_load_4d(sK + p * BN * 128, &args.tk, &k_full[0], p * 64, j_begin * BN, hk, b);
     }
   }
   if (warp == 9) {
@@ -281,7 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&args.tv);
-      const int zk = b * args.Hkv + hk;
       // K runs one tile ahead of V: a K stage frees as soon as both Q.K^T
       // products that read it are done, a V stage only after both P.V.
       // Q, the rel tables and K tile 0 were issued during setup.
@@ -295,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         const int key0 = (j_begin + jj) * BN;
         mbar_expect_tx(&k_full[s], L::kKVBytes);
         for (int p = 0; p < L::kPanels; ++p)
-          tma_load_3d(sK + s * L::kKVBytes + p * BN * 128, &args.tk, &k_full[s], p * 64, key0, zk);
+          tma_load_4d(sK + s * L::kKVBytes + p * BN * 128, &args.tk, &k_full[s], p * 64, key0, hk, b);
         k_issued = jj + 1;
       };
       auto load_v = [&](int jj) {
@@ -306,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         const int key0 = (j_begin + jj) * BN;
         mbar_expect_tx(&v_full[s], L::kKVBytes);
         for (int p = 0; p < L::kPanels; ++p)
-          tma_load_3d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, zk);
+          tma_load_4d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, hk, b);
         v_issued = jj + 1;
       };
       for (int jj = 1; jj < n_tiles && ok; ++jj) {
@@ -729,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 
     // epilogue: O / l -> bf16, rows past Tq are not stored
     const long long zq = (long long)b * args.Hq + h;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (zq * args.Tq + qi) * D;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (long long)b * args.sob + (long long)h * args.soh + qi * args.sot;
     if (n_tiles > 0 && ok) {
       if constexpr (kPSep)
         ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (n_tiles - 1) & 1, abort_v, args.err));
@@ -943,6 +942,13 @@ int tc_check(const Params& p, sdpa_dtype_t dtype) {
   if (p.Tkv < 1 || p.Tq < 1) return SDPA_ERR_UNSUPPORTED;
   if (p.B > 65535 || p.Hq > 65535) return SDPA_ERR_UNSUPPORTED;
   if (!al16(p.q) || !al16(p.k) || !al16(p.v) || !al16(p.out)) return SDPA_ERR_MISALIGNED;
+  // TMA: byte strides multiples of 16 and below 2^40
+  if (!strides_multiple_of(p, 8)) return SDPA_ERR_MISALIGNED;
+  {
+    const long long s[9] = {p.sqb, p.sqh, p.sqt, p.skb, p.skh, p.skt, p.svb, p.svh, p.svt};
+    for (long long x : s)
+      if (x >= (1LL << 38)) return SDPA_ERR_UNSUPPORTED;
+  }
   if (p.use_rel) {
     if (p.d != 64) return SDPA_ERR_UNSUPPORTED;
     const int kw = p.kw_n;
@@ -1008,9 +1014,10 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t rowb = (uint64_t)p.d * 2;
   const int BN = (p.use_rel && p.kw_n == 14) ? 112 : 128;
-  bool ok = make_tmap_3d(&a.tq, p.q, bf, 2, p.d, p.Tq, (uint64_t)p.B * p.Hq, rowb, rowb * p.Tq, 64, 128, true);
-  ok = ok && make_tmap_3d(&a.tk, p.k, bf, 2, p.d, p.Tkv, (uint64_t)p.B * p.Hkv, rowb, rowb * p.Tkv, 64, BN, true);
-  ok = ok && make_tmap_3d(&a.tv, p.v, bf, 2, p.d, p.Tkv, (uint64_t)p.B * p.Hkv, rowb, rowb * p.Tkv, 64, BN, true);
+  // (head_dim, token, head, batch) views with the tensors' own strides (bhsd, bshd, ...)
+  bool ok = make_tmap_4d(&a.tq, p.q, bf, p.d, p.Tq, p.Hq, p.B, 2 * p.sqt, 2 * p.sqh, 2 * p.sqb, 64, 128, true);
+  ok = ok && make_tmap_4d(&a.tk, p.k, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.skt, 2 * p.skh, 2 * p.skb, 64, BN, true);
+  ok = ok && make_tmap_4d(&a.tv, p.v, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.svt, 2 * p.svh, 2 * p.svb, 64, BN, true);
   if (p.use_rel) {
     const int kmax = p.kh_n > p.kw_n ? p.kh_n : p.kw_n;
     a.rel_n = ((2 * kmax - 1) + 15) / 16 * 16;
@@ -1020,6 +1027,7 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   }
   if (!ok) return cudaErrorInvalidValue;
   a.out = p.out;
+  a.sob = p.sob; a.soh = p.soh; a.sot = p.sot;
   a.lse = p.lse;
   a.mask = p.mask;
   a.msb = p.msb; a.msh = p.msh; a.msq = p.msq;

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p) {
   const long long i = (long long)blockIdx.x * kRowsPerCta + threadIdx.x;
   const bool valid = i < p.Tq;
   const long long zq = (long long)b * p.Hq + h;
-  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (zq * p.Tq + (valid ? i : 0)) * D16;
+  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, valid ? i : 0);
   float q[D16];
   bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
   bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
@@ -92,8 +92,8 @@ __global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p) {
   }
   const bool elementwise = p.mask_kind != SDPA_MASK_NONE;
   const long long mrow = (long long)b * p.msb + (long long)h * p.msh + i * p.msq;
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, 0);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, 0);
 
   float m = -INFINITY, l = 0.f, acc[D16];
 #pragma unroll
@@ -106,12 +106,12 @@ __global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p) {
     if (threadIdx.x < n) {
       const long long j = j0 + threadIdx.x;
       float f[D16];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * D16)), f);
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * D16) + 1), f + 8);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * p.skt)), f);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + j * p.skt) + 1), f + 8);
 #pragma unroll
       for (int c = 0; c < D16; c += 4) sk[threadIdx.x][c / 4] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * D16)), f);
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * D16) + 1), f + 8);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * p.svt)), f);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + j * p.svt) + 1), f + 8);
 #pragma unroll
       for (int c = 0; c < D16; c += 4) sv[threadIdx.x][c / 4] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
     }
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p) {
   o1.y = pack2(acc[10] * inv, acc[11] * inv);
   o1.z = pack2(acc[12] * inv, acc[13] * inv);
   o1.w = pack2(acc[14] * inv, acc[15] * inv);
-  uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (zq * p.Tq + i) * D16);
+  uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + o_off(p, b, h, i));
   orow[0] = o0;
   orow[1] = o1;
   if (p.lse) p.lse[zq * p.Tq + i] = l > 0.f ? m * kLn2 + logf(l) : -INFINITY;
@@ -204,16 +204,16 @@ __global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a)
   const long long zq = (long long)b * p.Hq + h;
   const long long j0 = (long long)part * a.chunk;
   const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + ((long long)b * p.Hkv + hk) * (long long)p.Tkv * D16;
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, 0);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, 0);
   for (int t = threadIdx.x; t < n; t += kSplitThreads) {
     float f[D16];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * D16)), f);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * D16) + 1), f + 8);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt)), f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt) + 1), f + 8);
 #pragma unroll
     for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * D16)), f);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * D16) + 1), f + 8);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt)), f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt) + 1), f + 8);
 #pragma unroll
     for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
   }
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl = p.scale * kLog2e;
   for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (zq * p.Tq + i) * D16;
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, i);
     float q[D16];
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a)
     const float val = den > 0.f ? num / den : 0.f;
     const float nb = __shfl_down_sync(0xffffffffu, val, 1);
     if (lane < D16 && (lane & 1) == 0) {
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + (zq * p.Tq + i) * D16;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + o_off(p, b, h, i);
       *reinterpret_cast<uint32_t*>(orow + lane) = pack2(val, nb);
     }
     if (lane == 0 && p.lse) p.lse[zq * p.Tq + i] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
@@ -367,6 +367,7 @@ int small_d_check(const Params& p, sdpa_dtype_t dtype) {
   const uintptr_t m = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
                       reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.out);
   if (m & 15) return SDPA_ERR_MISALIGNED;
+  if (!strides_multiple_of(p, 8)) return SDPA_ERR_MISALIGNED;  // 16-byte row loads / stores
   return SDPA_OK;
 }
 

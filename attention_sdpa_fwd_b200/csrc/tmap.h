@@ -47,4 +47,24 @@ inline bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType
   return r == CUDA_SUCCESS;
 }
 
+// 4-D map over a tensor of `elem_bytes` elements with dims {n0, n1, n2, n3}
+// (dim0 contiguous) and byte strides s1, s2, s3 of dims 1..3, in any order of
+// magnitude (e.g. head_dim, token, head, batch of a "bshd" tensor); box
+// {b0, b1, 1, 1}; 128-byte swizzle when asked.  Out-of-range elements of a box
+// read as zero.  Returns false if the driver rejects the map.
+inline bool make_tmap_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t n0,
+                         uint64_t n1, uint64_t n2, uint64_t n3, uint64_t s1, uint64_t s2, uint64_t s3,
+                         uint32_t b0, uint32_t b1, bool swizzle128) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {n0, n1, n2, n3};
+  cuuint64_t strides[3] = {s1, s2, s3};
+  cuuint32_t box[4] = {b0, b1, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace sdpa

@@ -26,7 +26,8 @@
  *     mask argument is an arbitrary additive array).
  *
  * Layout: every tensor is dense row-major "bhsd": q and out [B, Hq, Tq, d],
- * k and v [B, Hkv, Tkv, d], in the I/O dtype.  All data pointers are DEVICE
+ * k and v [B, Hkv, Tkv, d], in the I/O dtype -- except for sdpa_fwd_strided,
+ * which takes any batch / head / token strides (e.g. "bshd").  All data pointers are DEVICE
  * pointers owned by the caller; the library keeps no reference after a call
  * returns (it caches only TMA descriptors and a scratch buffer, see below).
  *
@@ -148,6 +149,39 @@ int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* out, sdpa_dty
                 const void* rel_pos_h, const void* rel_pos_w,
                 const int* q_hw, const int* k_hw,
                 float* lse, int path, cudaStream_t stream);
+
+/*
+ * sdpa_fwd_strided -- sdpa_fwd_ex on tensors with arbitrary batch, head and
+ * token strides, e.g. the "bshd" layout [B, T, H, d] that the Axon PR ("Add
+ * scaled_dot_product_attention", :axes option) takes by default, used in
+ * place (the PR's review asks to avoid the transposes to "bhsd").
+ *
+ * Each sdpa_strides_t holds the ELEMENT strides of the batch, head and token
+ * axes of one tensor; the head_dim axis is contiguous.  A NULL strides pointer
+ * means dense bhsd for that tensor: q and out {Hq*Tq*d, Tq*d, d}, k and v
+ * {Hkv*Tkv*d, Tkv*d, d}; bshd is {T*H*d, d, H*d}.  Strides must be positive
+ * (SDPA_ERR_INVALID_ARG otherwise).  The tensor-core path and the head_dim-16
+ * paths also need every stride to be a multiple of 8 elements for bf16 (their
+ * 16-byte TMA boxes and row loads); AUTO sends other problems to the exact
+ * kernel, an explicit path returns SDPA_ERR_MISALIGNED.  `out` must not
+ * overlap any input over their address spans (SDPA_ERR_INVALID_ARG).  lse,
+ * when given, is dense [B, Hq, Tq] as for sdpa_fwd_ex.
+ */
+typedef struct {
+  int64_t b;  /* batch stride (elements) */
+  int64_t h;  /* head stride  (elements) */
+  int64_t t;  /* token stride (elements) */
+} sdpa_strides_t;
+
+int sdpa_fwd_strided(const void* q, const sdpa_strides_t* q_strides,
+                     const void* k, const sdpa_strides_t* k_strides,
+                     const void* v, const sdpa_strides_t* v_strides,
+                     void* out, const sdpa_strides_t* out_strides,
+                     sdpa_dtype_t dtype, int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
+                     int mask_kind, const void* mask_ptr,
+                     const void* rel_pos_h, const void* rel_pos_w,
+                     const int* q_hw, const int* k_hw,
+                     float* lse, int path, cudaStream_t stream);
 
 /* The path AUTO would take for this problem (a non-negative sdpa_path_t), or a
    negative sdpa_status when the arguments are invalid.  Launches nothing;

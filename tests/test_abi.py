@@ -119,3 +119,25 @@ def test_binding_has_no_cpu_path():
     q = torch.zeros(1, 1, 4, 16)
     with pytest.raises(ValueError):
         S.sdpa(q, q, q)
+
+
+def test_strided_entry_validates_strides(L):
+    """sdpa_fwd_strided rejects non-positive strides and an output whose
+    address span overlaps an input's, before any launch."""
+    B, H, T, d = 1, 2, 8, 64
+    q, k, v, out = 4096, 4096 * 64, 4096 * 128, 4096 * 256  # fake, 16-byte aligned, disjoint
+    base = dict(dtype=S.SDPA_BF16, B=B, Hq=H, Hkv=H, Tq=T, Tkv=T, d=d, scale=0.1, mask_kind=0, mask_ptr=None,
+                rel_pos_h=None, rel_pos_w=None, q_hw=None, k_hw=None, lse=None, path=0, stream=None)
+
+    def call(qs=None, ks=None, vs=None, os_=None, out_ptr=out):
+        return S.sdpa_fwd_strided(q, qs, k, ks, v, vs, out_ptr, os_, **base)
+
+    for bad in ((0, 64, 128), (1024, -64, 128), (1024, 64, 0)):
+        assert call(qs=bad) == -1
+        assert call(ks=bad) == -1
+        assert call(os_=bad) == -1
+    # bshd out whose span reaches into q
+    assert call(os_=(T * H * d, d, H * d), out_ptr=q + 64) == -1
+    # unsupported head_dim is reported as such whatever the strides
+    b2 = dict(base, d=48)
+    assert S.sdpa_fwd_strided(q, None, k, None, v, None, out, None, **b2) == -2
