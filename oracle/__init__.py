@@ -144,3 +144,30 @@ def sdpa(q, k, v, scale: float, *, mask_kind: int = MASK_NONE, offset: int = 0,
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return OracleResult(out=out, lse=lse, weights=w)
+
+
+def merge(outs: Sequence, lses: Sequence):
+    """Combine attention results over disjoint key subsets into the result
+    over their union, in fp64.
+
+    Part i holds ``out_i = sum_j p_ij v_j / l_i`` and ``lse_i = m_i + log l_i``
+    over its own keys (the natural-log sum-exp of its score rows, -inf when
+    no key is visible).  Over the union the normaliser is
+    ``L = log sum_i exp(lse_i)`` and every part's unnormalised sum is
+    ``exp(lse_i) * out_i``, so ``out = sum_i exp(lse_i - L) * out_i``; a row
+    with no visible key anywhere gives ``out = 0``, ``L = -inf``.  This is the
+    split-key combination the Axon PR's attention reaches by summing the
+    softmax numerators of all keys (PR description: softmax(Q.K^T*scale+mask).V
+    over the whole key axis).  Inputs: sequences of arrays [..., d] and [...].
+    Returns (out, lse) as float64 arrays."""
+    o = np.stack([_f64(x) for x in outs])            # [n, ..., d]
+    s = np.stack([_f64(x) for x in lses])            # [n, ...]
+    top = np.max(s, axis=0)                          # [...]
+    finite = np.isfinite(top)
+    shifted = np.where(finite[None], s - np.where(finite, top, 0.0)[None], -np.inf)
+    w = np.exp(shifted)                              # exp(lse_i - top), 0 for -inf parts
+    tot = np.sum(w, axis=0)
+    lse = np.where(finite, top + np.log(np.where(finite, tot, 1.0)), -np.inf)
+    wn = np.where(finite[None], w / np.where(finite, tot, 1.0)[None], 0.0)
+    out = np.sum(wn[..., None] * o, axis=0)
+    return out, lse
