@@ -26,7 +26,7 @@ STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
           -6: "SDPA_ERR_CAPACITY"}
 
 # Every symbol include/sdpa.h declares.
-EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_select_path", "sdpa_fwd_host",
+EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_merge", "sdpa_select_path", "sdpa_fwd_host",
            "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_strerror", "sdpa_version")
 
 
@@ -61,13 +61,14 @@ def lib():
         L.sdpa_fwd.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
         L.sdpa_fwd_ex.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
         L.sdpa_fwd_host.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+        L.sdpa_merge.argtypes = [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]
         L.sdpa_fwd_strided.argtypes = [_vp] * 8 + [_i32] * 7 + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
         L.sdpa_select_path.argtypes = _COMMON + [_i32, _vp, _vp, _vp, _vp, _vp]
         L.sdpa_fwd_split_kv_static.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp]
         L.sdpa_last_device_error.argtypes = [_vp]
         L.sdpa_strerror.argtypes = [_i32]
         L.sdpa_strerror.restype = ctypes.c_char_p
-        for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_fwd_host", "sdpa_select_path",
+        for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_merge", "sdpa_fwd_host", "sdpa_select_path",
                      "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_version"):
             getattr(L, name).restype = _i32
         _lib = L
@@ -99,6 +100,13 @@ def sdpa_fwd_strided(q, q_strides, k, k_strides, v, v_strides, out, out_strides,
     return lib().sdpa_fwd_strided(q, st(q_strides), k, st(k_strides), v, st(v_strides), out, st(out_strides),
                                   dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr, rel_pos_h, rel_pos_w,
                                   _hw(q_hw), _hw(k_hw), lse, path, stream)
+
+
+def sdpa_merge(outs, lses, nparts, out, lse, dtype, B, Hq, Tq, d, stream) -> int:
+    """outs / lses: sequences of device pointers (ints)."""
+    po = (ctypes.c_void_p * len(outs))(*outs)
+    pl = (ctypes.c_void_p * len(lses))(*lses)
+    return lib().sdpa_merge(po, pl, nparts, out, lse, dtype, B, Hq, Tq, d, stream)
 
 
 def sdpa_fwd_host(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
@@ -210,3 +218,28 @@ def sdpa(q, k, v, scale: Optional[float] = None, *, mask_kind: int = MASK_NONE, 
     if rc != 0:
         raise SdpaError(rc, what)
     return out
+
+
+def merge(outs, lses, out=None, lse=None, stream=None):
+    """Combine attention results over disjoint key subsets (sdpa_merge).
+
+    outs: sequence of [B, Hq, Tq, d] CUDA tensors (dense, same dtype); lses:
+    matching [B, Hq, Tq] float32 tensors as written by ``sdpa(..., lse=)``.
+    Returns (out, lse); ``out`` may be ``outs[0]`` (in place)."""
+    import torch
+    o0 = outs[0]
+    for t in list(outs) + list(lses):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("merge takes dense CUDA tensors only")
+    B, Hq, Tq, d = o0.shape
+    if out is None:
+        out = torch.empty_like(o0)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), device=o0.device, dtype=torch.float32)
+    st = stream if stream is not None else torch.cuda.current_stream(o0.device)
+    with torch.cuda.device(o0.device):
+        rc = sdpa_merge([t.data_ptr() for t in outs], [t.data_ptr() for t in lses], len(outs), out.data_ptr(),
+                        lse.data_ptr(), _dtype_code(o0), B, Hq, Tq, d, st.cuda_stream)
+    if rc != 0:
+        raise SdpaError(rc, "sdpa_merge")
+    return out, lse

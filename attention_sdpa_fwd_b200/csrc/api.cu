@@ -298,6 +298,32 @@ extern "C" int sdpa_fwd_strided(const void* q, const sdpa_strides_t* q_strides, 
   return run(pr, path, stream);
 }
 
+extern "C" int sdpa_merge(const void* const* outs, const float* const* lses, int nparts, void* out, float* lse,
+                          sdpa_dtype_t dtype, int B, int Hq, int Tq, int d, cudaStream_t stream) {
+  if (dtype != SDPA_F32 && dtype != SDPA_BF16) return SDPA_ERR_INVALID_ARG;
+  if (nparts < 1 || nparts > kMaxMergeParts || outs == nullptr || lses == nullptr) return SDPA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Tq < 0) return SDPA_ERR_INVALID_ARG;
+  if (!(d == 16 || d == 64 || d == 128)) return SDPA_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * Hq * Tq;
+  if (rows == 0) return SDPA_OK;
+  if (out == nullptr) return SDPA_ERR_INVALID_ARG;
+  const size_t esz = dtype == SDPA_F32 ? 4 : 2;
+  const size_t no = (size_t)rows * d * esz, nl = (size_t)rows * 4;
+  if (!aligned(out, 16) || (lse && !aligned(lse, 4))) return SDPA_ERR_MISALIGNED;
+  for (int i = 0; i < nparts; ++i) {
+    if (outs[i] == nullptr || lses[i] == nullptr) return SDPA_ERR_INVALID_ARG;
+    if (!aligned(outs[i], 16) || !aligned(lses[i], 4)) return SDPA_ERR_MISALIGNED;
+    // out may be part 0 exactly (in place); no other overlap
+    if (!(i == 0 && outs[i] == out) && overlaps(out, no, outs[i], no)) return SDPA_ERR_INVALID_ARG;
+    if (overlaps(out, no, lses[i], nl)) return SDPA_ERR_INVALID_ARG;
+    if (lse && !(i == 0 && lses[i] == lse) && overlaps(lse, nl, lses[i], nl)) return SDPA_ERR_INVALID_ARG;
+    if (lse && overlaps(lse, nl, outs[i], no)) return SDPA_ERR_INVALID_ARG;
+  }
+  if (lse && overlaps(lse, nl, out, no)) return SDPA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_merge(outs, lses, nparts, out, lse, dtype, rows, d, stream);
+  return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
+
 extern "C" int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
                         int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
                         const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,

@@ -102,4 +102,9 @@ int split_kv_static(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
 int num_sms();
 cudaError_t launch_tc(const Params& p, cudaStream_t stream);
 
+// Parts sdpa_merge combines at most.
+constexpr int kMaxMergeParts = 16;
+cudaError_t launch_merge(const void* const* outs, const float* const* lses, int n, void* out, float* lse,
+                         sdpa_dtype_t dtype, long long rows, int d, cudaStream_t stream);
+
 }  // namespace sdpa

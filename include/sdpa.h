@@ -183,6 +183,28 @@ int sdpa_fwd_strided(const void* q, const sdpa_strides_t* q_strides,
                      const int* q_hw, const int* k_hw,
                      float* lse, int path, cudaStream_t stream);
 
+/*
+ * sdpa_merge -- combine attention results over disjoint key subsets of the
+ * same queries into the result over their union, e.g. a long key axis run
+ * chunk by chunk through sdpa_fwd_ex with its lse output.  Part i gives
+ * out_i [B, Hq, Tq, d] (I/O dtype, dense bhsd) and lse_i [B, Hq, Tq] (float,
+ * natural-log sum-exp of its score rows, -inf where it saw no key).  Writes
+ *     lse = L = log sum_i exp(lse_i),   out = sum_i exp(lse_i - L) * out_i
+ * -- the softmax numerators of every key summed, as attention over the whole
+ * key axis does (Axon PR "Add scaled_dot_product_attention": softmax(Q.K^T *
+ * scale + mask).V).  A row whose parts are all -inf gets zeros and -inf.
+ *   outs, lses : HOST arrays of `nparts` DEVICE pointers, 1 <= nparts <= 16.
+ *   out        : device output; may be outs[0] (in place), must not overlap
+ *                any other part.  16-byte aligned, as must every outs[i].
+ *   lse        : device float output or NULL; may be lses[0].
+ * d must be 16, 64 or 128.  Errors: SDPA_ERR_INVALID_ARG (counts, NULLs,
+ * overlap), SDPA_ERR_UNSUPPORTED (d), SDPA_ERR_MISALIGNED.  Asynchronous on
+ * `stream`.
+ */
+int sdpa_merge(const void* const* outs, const float* const* lses, int nparts,
+               void* out, float* lse, sdpa_dtype_t dtype, int B, int Hq, int Tq, int d,
+               cudaStream_t stream);
+
 /* The path AUTO would take for this problem (a non-negative sdpa_path_t), or a
    negative sdpa_status when the arguments are invalid.  Launches nothing;
    pointers are only checked for NULL and alignment. */

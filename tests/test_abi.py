@@ -141,3 +141,14 @@ def test_strided_entry_validates_strides(L):
     # unsupported head_dim is reported as such whatever the strides
     b2 = dict(base, d=48)
     assert S.sdpa_fwd_strided(q, None, k, None, v, None, out, None, **b2) == -2
+
+
+def test_merge_validates_on_host(L):
+    o, l = [4096, 8192], [65536, 131072]  # fake, aligned, disjoint device addresses
+    ok = dict(dtype=S.SDPA_BF16, B=1, Hq=2, Tq=8, d=64, stream=None)
+    assert S.sdpa_merge(o, l, 0, 1 << 20, 1 << 21, **ok) == -1          # no parts
+    assert S.sdpa_merge(o * 9, l * 9, 17, 1 << 20, 1 << 21, **ok) == -1  # too many parts
+    assert S.sdpa_merge(o, l, 2, 1 << 20, 1 << 21, **dict(ok, d=48)) == -2
+    assert S.sdpa_merge(o, l, 2, (1 << 20) + 8, 1 << 21, **ok) == -3     # out not 16-byte aligned
+    assert S.sdpa_merge(o, l, 2, 8192 + 64, 1 << 21, **ok) == -1         # out overlaps part 1
+    assert S.sdpa_merge(o, l, 2, 1 << 20, None, **dict(ok, Tq=0)) == 0   # nothing to do
