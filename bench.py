@@ -259,6 +259,34 @@ def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, w
                 set_bytes=per_set)
 
 
+def time_graph(S, spec: W.Spec, device, launches: int = 40, reps: int = 5):
+    """Per-launch device time from CUDA-graph replays of `launches` back-to-back
+    launches (rotating input sets): strips the host launch overhead that
+    dominates per-launch events for the microsecond-sized workloads."""
+    per_set = spec.bytes()
+    nsets = min(16, max(2, math.ceil(2 * L2_BYTES / max(per_set, 1))))
+    sets = make_device_sets(spec, device, nsets, seed_base=spec.seed)
+    side = torch.cuda.Stream(device)
+    with torch.cuda.stream(side):
+        for i in range(3):
+            launch(S, spec, sets[i % nsets], side, 0)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(launches):
+            launch(S, spec, sets[i % nsets], side, 0)
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / (reps * launches)
+
+
 def time_e2e(S, spec: W.Spec, device, steps: int, warmup: int):
     """Same forward through the host-buffer C entry point: pinned host inputs,
     H2D copies, kernel, D2H copy of the output, all inside the timed region."""
@@ -305,11 +333,15 @@ def time_e2e(S, spec: W.Spec, device, steps: int, warmup: int):
     return ms, h2d, d2h
 
 
+_WL_CACHE = {}
+
+
 def cpu_oracle_sample(spec: W.Spec, budget_s: float = 12.0):
     """Time the fp64 oracle on the host cores on a bounded row sample."""
     import oracle
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    wl = W.make(spec)
+    if spec.name not in _WL_CACHE:
+        _WL_CACHE[spec.name] = W.make(spec)
+    wl = _WL_CACHE[spec.name]
     kw = dict(mask_kind=spec.mask_kind, offset=spec.offset, window=spec.window)
     if spec.mask_kind in (W.MASK_FLOAT, W.MASK_BOOL):
         kw["mask"] = wl.mask
@@ -407,8 +439,13 @@ def run_ours(args):
                 continue
             rr = time_workload(S, sp, device, max(3, args.steps // 4), 3, 0, 1)
             lm = sum(rr["launch_ms"]) / len(rr["launch_ms"])
-            per_config[name] = dict(ms=lm, tflops=sp.flops() / (lm * 1e-3) / 1e12,
-                                    gbs=sp.bytes() / (lm * 1e-3) / 1e9)
+            gm = time_graph(S, sp, device)
+            hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+            bf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            per_config[name] = dict(ms=lm, graph_ms=gm, tflops=sp.flops() / (gm * 1e-3) / 1e12,
+                                    gbs=sp.bytes() / (gm * 1e-3) / 1e9,
+                                    frac_bf16=sp.flops() / (gm * 1e-3) / 1e12 / bf,
+                                    frac_hbm=sp.bytes() / (gm * 1e-3) / 1e9 / hbm)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -463,7 +500,8 @@ def run_reference(args):
     spec = W.SPECS[args.workload]
     vals = []
     info = None
-    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # about 150 s of oracle work in all, whatever --steps / --warmup ask for
+    budget = max(0.1, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
         info = cpu_oracle_sample(spec, budget_s=budget)
         if i >= args.warmup:
