@@ -109,7 +109,7 @@ struct Layout {
   static constexpr int oV = oK + NS * kKVBytes;
   static constexpr int oRel = oV + NS * kKVBytes;
   static constexpr int oBar = oRel + kRelRows * 256 * 4;
-  static constexpr int kBars = 4 * NS + 14;
+  static constexpr int kBars = 4 * NS + 20;
   static constexpr int kTotal = oBar + kBars * 8 + 32;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -153,6 +153,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   // softmax t has read S_t(j), before P_t(j) exists.  At head_dim 128, P_t
   // overwrites S_t and the next Q.K^T waits for P_t.V.
   constexpr bool kPSep = (D == 64);
+  // head_dim 128 with 64-key tiles: each query tile gets two 64-column S
+  // buffers at [128t, 128t+64) and [128t+64, 128t+128) (O_t at 256+128t), and
+  // P_t(j) is written over the first half of the S buffer it was read from.
+  // S_t(j+2) goes into that buffer right after O_t += P_t(j).V_j (in issue
+  // order), so the next score tile is always computed one tile ahead.
+  constexpr bool kSDB = (D == 128 && BN == 64);
   constexpr bool kRwInSmem = KW >= 32;  // large key-grid width: rel_w re-read per tile
   constexpr int kRwSwz = KW >= 64 ? 15 : 7;  // float4-index XOR swizzle of those rows (conflict-free)
   extern __shared__ uint8_t smem_raw[];
@@ -177,6 +183,15 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   uint64_t* fin = q_full + 9;            // last commit before TMEM release
   uint64_t* s_free = q_full + 10;        // [2]   softmax t read S_t (128 arrivals) -> MMA   (kPSep)
   uint64_t* o_ready = q_full + 12;       // [2]   MMA commit after each O_t += P_t V         (kPSep)
+  // kSDB: O_t += P_t(j).V_j commits o_ready[t] for even j and o_odd[t] for odd
+  // j, so that each barrier is at most one phase from any wait on it
+  uint64_t* o_odd = q_full + 14;         // [2]
+  // kSDB: likewise S_t(j) completes s_full[t] / s_odd[t] and P_t(j) arrives on
+  // p_full[t] / p_odd[t] by the parity of j -- with two S buffers either side
+  // can run a tile ahead, and a single barrier could then be two phases ahead
+  // of its waiter
+  uint64_t* s_odd = q_full + 16;         // [2]
+  uint64_t* p_odd = q_full + 18;         // [2]   (128 arrivals)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + L::kBars);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
 
@@ -227,6 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     mbar_init(rel_read, 2 * kRowsPerTile);
     mbar_init(&s_free[0], kRowsPerTile);
     mbar_init(&s_free[1], kRowsPerTile);
+    mbar_init(&p_odd[0], kRowsPerTile);
+    mbar_init(&p_odd[1], kRowsPerTile);
     fence_mbar_init();
     if (n_tiles > 0) {
       // Q (and the rel tables) and the first K tile go out before the TMEM
@@ -308,11 +325,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           tma_load_4d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, hk, b);
         v_issued = jj + 1;
       };
+      constexpr int kAhead = kSDB ? 2 : 1;  // K tiles loaded ahead of V (the MMA issues S two tiles ahead in kSDB)
       for (int jj = 1; jj < n_tiles && ok; ++jj) {
         load_k(jj);
-        if (ok) load_v(jj - 1);
+        if (ok && jj >= kAhead) load_v(jj - kAhead);
       }
-      if (ok) load_v(n_tiles - 1);
+      for (int jv = max(0, n_tiles - kAhead); jv < n_tiles && ok; ++jv) load_v(jv);
       if (!ok) {
         // abandoned: let the copies already in flight land before the CTA exits
         mbar_wait(q_full, 0, nullptr, args.err);
@@ -335,10 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       const uint64_t dk = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dv = sdesc_sw128(smem_u32(sV), BN * 128, 1024);
       bool ok = wait_x(mbar_wait(q_full, 0, abort_v, args.err));
-      auto qk = [&](int t, int s) {
+      auto qk = [&](int t, int s, int buf = 0) {
         const uint64_t a0 = dq + (uint64_t)((t * L::kQBytes) >> 4);
         const uint64_t b0 = dk + (uint64_t)((s * L::kKVBytes) >> 4);
-        const uint32_t d_tm = tbase + t * 128;
+        const uint32_t d_tm = tbase + t * 128 + buf * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = ((kk >> 2) * (kRowsPerTile * 128) + (kk & 3) * 32) >> 4;
@@ -346,10 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           mma_ss_x(d_tm, a0 + ao, b0 + bo, id_qk, kk > 0);
         }
       };
-      auto pv = [&](int t, int s, bool first) {
+      auto pv = [&](int t, int s, bool first, int buf = 0) {
         const uint64_t b0 = dv + (uint64_t)((s * L::kKVBytes) >> 4);
         const uint32_t d_tm = tbase + 256 + t * D;
-        const uint32_t a_tm = kPSep ? tbase + 384 + t * 64 : tbase + t * 128;
+        const uint32_t a_tm = kPSep ? tbase + 384 + t * 64 : tbase + t * 128 + buf * 64;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           mma_ts_x(d_tm, a_tm + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (!first) || kk > 0);
@@ -379,7 +397,49 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         mma_commit_x(&s_full[1]);
         mma_commit_x(&k_empty[0]);
       }
-      if constexpr (kPSep) {
+      if (kSDB && ok && n_tiles > 1) {
+        ok = wait_x(mbar_wait(&k_full[1], 0, abort_v, args.err));
+        if (ok) {
+          tc_fence_after();
+          qk(0, 1, 1);
+          mma_commit_x(&s_odd[0]);
+          qk(1, 1, 1);
+          mma_commit_x(&s_odd[1]);
+          mma_commit_x(&k_empty[1]);
+        }
+      }
+      if constexpr (kSDB) {
+        // O_t += P_t(j).V_j, then S_t(j+2) into the buffer P_t(j) was read from
+        for (int jj = 0; jj < n_tiles && ok; ++jj) {
+          const int s = jj % NS, buf = jj & 1;
+          const bool more = jj + 2 < n_tiles;
+          const int s2 = (jj + 2) % NS;
+          ok = wait_x(mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err));
+          if (ok) ok = wait_x(mbar_wait(buf ? &p_odd[0] : &p_full[0], (jj >> 1) & 1, abort_v, args.err));
+          if (!ok) break;
+          tc_fence_after();
+          pv(0, s, jj == 0, buf);
+          mma_commit_x(jj & 1 ? &o_odd[0] : &o_ready[0]);
+          if (more) {
+            ok = wait_x(mbar_wait(&k_full[s2], ((jj + 2) / NS) & 1, abort_v, args.err));
+            if (!ok) break;
+            tc_fence_after();
+            qk(0, s2, buf);
+            mma_commit_x(buf ? &s_odd[0] : &s_full[0]);
+          }
+          ok = wait_x(mbar_wait(buf ? &p_odd[1] : &p_full[1], (jj >> 1) & 1, abort_v, args.err));
+          if (!ok) break;
+          tc_fence_after();
+          pv(1, s, jj == 0, buf);
+          mma_commit_x(jj & 1 ? &o_odd[1] : &o_ready[1]);
+          mma_commit_x(&v_empty[s]);
+          if (more) {
+            qk(1, s2, buf);
+            mma_commit_x(buf ? &s_odd[1] : &s_full[1]);
+            mma_commit_x(&k_empty[s2]);
+          }
+        }
+      } else if constexpr (kPSep) {
         // A and B alternate: S_A(j+1), O_A += P_A(j).V_j, S_B(j+1), O_B += P_B(j).V_j
         for (int jj = 0; jj < n_tiles && ok; ++jj) {
           const int s = jj % NS;
@@ -458,9 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     const int row = t * kRowsPerTile + lr;   // row within the CTA
     const long long qi = (long long)q0 + row;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tbase + lane_off + t * 128;
+    const uint32_t s_base = tbase + lane_off + t * 128;
     const uint32_t o_addr = tbase + lane_off + 256 + t * D;
-    const uint32_t p_addr = kPSep ? tbase + lane_off + 384 + t * 64 : s_addr;
+    const uint32_t p_fixed = tbase + lane_off + 384 + t * 64;  // kPSep
     bool ok = true;
     float* relh_s = sRel;                   // [kRelHMax][256]
     float* relw_s = sRel + kRelHMax * 256;  // [KW][256], or [256][KW] (swizzled) when read as float4 per tile
@@ -531,9 +591,15 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     float m_run = -INFINITY, l_run = 0.f;
     for (int jj = 0; jj < n_tiles && ok; ++jj) {
       const int j0 = (j_begin + jj) * BN;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], jj & 1, abort_v, args.err));
+      if constexpr (kSDB)
+        ok = __all_sync(0xffffffffu, mbar_wait(jj & 1 ? &s_odd[t] : &s_full[t], (jj >> 1) & 1, abort_v, args.err));
+      else
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], jj & 1, abort_v, args.err));
       if (!ok) break;
       tc_fence_after();
+      // this tile's S columns (and, unless P has its own, where P goes)
+      const uint32_t s_addr = s_base + (kSDB ? (jj & 1) * 64 : 0);
+      const uint32_t p_addr = kPSep ? p_fixed : s_addr;
       uint32_t sr[BN];
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -707,7 +773,20 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           tc_fence_after();
         }
       }
-      if (jj > 0 && __any_sync(0xffffffffu, need)) {
+      const bool rescale = jj > 0 && __any_sync(0xffffffffu, need);
+      if constexpr (kSDB) {
+        // P_t(j) overwrites a buffer whose last reader, P_t(j-2).V, completed
+        // before S_t(j) (same commit); only a rescale of O_t waits for
+        // O_t += P_t(j-1).V, on the barrier of its parity: P_t(j-3).V is done
+        // and P_t(j+1).V cannot be, so that barrier is within one phase
+        if (rescale) {
+          const int x = jj - 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(x & 1 ? &o_odd[t] : &o_ready[t], (x >> 1) & 1, abort_v, args.err));
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
+      if (rescale) {
         // O_t row *= alpha (warp-collective; alpha is 1 where the max did not move)
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -723,15 +802,20 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       for (int c0 = 0; c0 < BN / 2; c0 += 8) tmem_st8p(p_addr + c0, pk + c0);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      mbar_arrive(kSDB && (jj & 1) ? &p_odd[t] : &p_full[t]);
     }
 
     // epilogue: O / l -> bf16, rows past Tq are not stored
     const long long zq = (long long)b * args.Hq + h;
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (long long)b * args.sob + (long long)h * args.soh + qi * args.sot;
     if (n_tiles > 0 && ok) {
-      if constexpr (kPSep)
+      if constexpr (kSDB) {
+        // the last two P.V may both be in flight, one on each parity's barrier
+        for (int x = max(0, n_tiles - 2); x < n_tiles && ok; ++x)
+          ok = __all_sync(0xffffffffu, mbar_wait(x & 1 ? &o_odd[t] : &o_ready[t], (x >> 1) & 1, abort_v, args.err));
+      } else if constexpr (kPSep) {
         ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (n_tiles - 1) & 1, abort_v, args.err));
+      }
       else
         ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, abort_v, args.err));
       tc_fence_after();
@@ -966,7 +1050,14 @@ int tc_check(const Params& p, sdpa_dtype_t dtype) {
 // Units (256-row query blocks of one (batch, head)) of a problem.
 long long nblk_of(const Params& p, int nqblk) { return (long long)nqblk * p.Hq * p.B; }
 // Key-tile width of the kernel instance the problem dispatches to.
-int BN_of(const Params& p) { return (p.use_rel && p.kw_n == 14) ? 112 : 128; }
+// head_dim 128 with a mask tensor runs 64-key tiles with two S buffers per
+// query tile (measured faster there: 3.32 ms against 3.97 ms on the 8192-token
+// float-mask problem); without one, 128-key tiles (1.09 ms against 1.22 ms causal).
+int BN_of(const Params& p) {
+  if (p.use_rel) return p.kw_n == 14 ? 112 : 128;
+  const bool tensor_mask = p.mask_kind == SDPA_MASK_ADD_FLOAT || p.mask_kind == SDPA_MASK_BOOL;
+  return (p.d == 128 && tensor_mask) ? 64 : 128;
+}
 
 // Picks how many units run whole (first) and into how many parts each of the
 // rest is split, minimising the modelled time on nsm SMs with one CTA each.
@@ -1013,7 +1104,7 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   memset(&a, 0, sizeof(a));
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t rowb = (uint64_t)p.d * 2;
-  const int BN = (p.use_rel && p.kw_n == 14) ? 112 : 128;
+  const int BN = BN_of(p);  // the K/V box must match the kernel instance's key tile
   // (head_dim, token, head, batch) views with the tensors' own strides (bhsd, bshd, ...)
   bool ok = make_tmap_4d(&a.tq, p.q, bf, p.d, p.Tq, p.Hq, p.B, 2 * p.sqt, 2 * p.sqh, 2 * p.sqb, 64, 128, true);
   ok = ok && make_tmap_4d(&a.tk, p.k, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.skt, 2 * p.skh, 2 * p.skb, 64, BN, true);
@@ -1063,6 +1154,7 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   dim3 grid((unsigned)(a.n_full + n_split_units * a.n_split), 1u, 1u);
   if (!p.use_rel) {
     if (p.d == 64) return dispatch_mask<64, 128, 0, 3>(mk, a, grid, stream);
+    if (BN_of(p) == 64) return dispatch_mask<128, 64, 0, 4>(mk, a, grid, stream);
     return dispatch_mask<128, 128, 0, 2>(mk, a, grid, stream);
   }
   switch (p.kw_n) {
