@@ -83,6 +83,12 @@ CASES = [
        mask_neg_inf_frac=0.2, mask_heads=2, seed=34),
     S_("bool_bf16_d128_aligned", BF16, 1, 2, 2, 260, 272, 128, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.5,
        mask_heads=1, seed=35),
+    # head_dim 128 with a mask tensor runs 64-key tiles with two score buffers:
+    # a single key tile, and an odd number of tiles with a ragged last one
+    S_("float_bf16_d128_one_tile", BF16, 1, 2, 1, 70, 50, 128, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=1, seed=36),
+    S_("float_bf16_d128_odd_tiles", BF16, 2, 3, 3, 200, 300, 128, mask_kind=W.MASK_FLOAT, mask_std=2.0,
+       mask_neg_inf_frac=0.1, mask_heads=3, seed=37),
 ]
 CASE_IDS = [c.name for c in CASES]
 
