@@ -25,6 +25,10 @@
 // exact kernel does).
 #include <math.h>
 
+#include <mutex>
+
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -358,6 +362,185 @@ __global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a)
   if (threadIdx.x == 0) a.ws_cnt[zq] = 0;  // ready for the next launch
 }
 
+// ------------------------------------------------------------------ split_kv over a cluster
+// The same split of the key axis, with the parts of one (batch, head) in one
+// thread-block cluster: each CTA leaves its partial (O, m, l) per query row
+// in its own shared memory, and CTA 0 of the cluster merges them through
+// distributed shared memory -- no global workspace, fence or ticket, so the
+// whole forward is one pass over K and V.  Used when the key axis fits in 8
+// parts of at most 512 keys.
+constexpr int kClusterMax = 8;      // portable cluster size
+constexpr int kClusterChunk = 512;  // keys per CTA (at most)
+constexpr int kRowsMax = 64;        // query rows the partial area holds
+constexpr int kPartStride = 20;     // floats per row partial: 16 O, m, l, pad
+
+struct ClusterArgs {
+  Params p;
+  int ncl;    // parts = cluster size
+  int chunk;  // keys per part
+};
+
+__global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(ClusterArgs a) {
+  namespace cg = cooperative_groups;
+  const Params& p = a.p;
+  extern __shared__ float4 cl_smem[];
+  float4 (*sk)[D16 / 4] = reinterpret_cast<float4 (*)[D16 / 4]>(cl_smem);
+  float4 (*sv)[D16 / 4] = reinterpret_cast<float4 (*)[D16 / 4]>(cl_smem + kClusterChunk * (D16 / 4));
+  float* part_s = reinterpret_cast<float*>(cl_smem + 2 * kClusterChunk * (D16 / 4));  // [Tq][kPartStride]
+  cg::cluster_group cluster = cg::this_cluster();
+  const int part = (int)cluster.block_rank(), h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.group;
+  const long long zq = (long long)b * p.Hq + h;
+  const long long j0 = (long long)part * a.chunk;
+  const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, 0);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, 0);
+  for (int t = threadIdx.x; t < n; t += kSplitThreads) {
+    float f[D16];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt)), f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt) + 1), f + 8);
+#pragma unroll
+    for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt)), f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt) + 1), f + 8);
+#pragma unroll
+    for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float sl = p.scale * kLog2e;
+  for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, i);
+    float q[D16];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
+    const long long mrow = (long long)b * p.msb + (long long)h * p.msh + (long long)i * p.msq;
+    // this lane's keys (lane, lane + 32, ...), in two halves of eight to
+    // bound the registers: scores, running max, then the sums
+    float m = -INFINITY, l = 0.f, acc[D16];
+#pragma unroll
+    for (int c = 0; c < D16; ++c) acc[c] = 0.f;
+#pragma unroll
+    for (int half = 0; half < kClusterChunk / 256; ++half) {
+      float sc[8];
+      float cm = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = lane + 32 * (half * 8 + u);
+        float x = -INFINITY;
+        if (t < n) {
+          x = 0.f;
+#pragma unroll
+          for (int c = 0; c < D16; c += 4) {
+            const float4 k4 = sk[t][(c / 4) ^ ((t >> 1) & 3)];
+            x = fmaf(q[c], k4.x, fmaf(q[c + 1], k4.y, fmaf(q[c + 2], k4.z, fmaf(q[c + 3], k4.w, x))));
+          }
+          x = x * sl + mask_term(p, mrow, i, j0 + t);
+        }
+        sc[u] = x;
+        cm = fmaxf(cm, x);
+      }
+      if (cm == -INFINITY) continue;
+      if (cm > m) {
+        const float corr = sm100::ex2_approx(m - cm);  // 0 when m == -inf
+        l *= corr;
+#pragma unroll
+        for (int c = 0; c < D16; ++c) acc[c] *= corr;
+        m = cm;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = lane + 32 * (half * 8 + u);
+        const float pj = sm100::ex2_approx(sc[u] - m);  // 0 for -inf
+        l += pj;
+        if (t < n) {
+#pragma unroll
+          for (int c = 0; c < D16; c += 4) {
+            const float4 v4 = sv[t][(c / 4) ^ ((t >> 1) & 3)];
+            acc[c] = fmaf(pj, v4.x, acc[c]);
+            acc[c + 1] = fmaf(pj, v4.y, acc[c + 1]);
+            acc[c + 2] = fmaf(pj, v4.z, acc[c + 2]);
+            acc[c + 3] = fmaf(pj, v4.w, acc[c + 3]);
+          }
+        }
+      }
+    }
+    // combine the 32 lanes: max, sum, and the 16 columns by a butterfly
+    // reduce-scatter (lane pair (2k, 2k+1) ends with column bits 4..1 of the lane)
+    float M = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = (m == -INFINITY) ? 0.f : sm100::ex2_approx(m - M);
+    l *= w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+    for (int c = 0; c < D16; ++c) acc[c] *= w;
+    float r8[8], r4[4], r2[2], r1;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const bool hi = lane & 16;
+      r8[k] = (hi ? acc[k + 8] : acc[k]) + __shfl_xor_sync(0xffffffffu, hi ? acc[k] : acc[k + 8], 16);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool hi = lane & 8;
+      r4[k] = (hi ? r8[k + 4] : r8[k]) + __shfl_xor_sync(0xffffffffu, hi ? r8[k] : r8[k + 4], 8);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const bool hi = lane & 4;
+      r2[k] = (hi ? r4[k + 2] : r4[k]) + __shfl_xor_sync(0xffffffffu, hi ? r4[k] : r4[k + 2], 4);
+    }
+    {
+      const bool hi = lane & 2;
+      r1 = (hi ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, hi ? r2[0] : r2[1], 2);
+    }
+    r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+    float* pr = part_s + i * kPartStride;
+    if ((lane & 1) == 0) pr[((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = r1;
+    if (lane == 0) {
+      pr[16] = M;
+      pr[17] = l;
+    }
+  }
+  // every part's partials are in its shared memory; CTA 0 of the cluster
+  // reads them all (distributed shared memory) and writes the rows
+  cluster.sync();
+  if (part == 0) {
+    for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
+      float Mk = -INFINITY, lk = 0.f;
+      if (lane < a.ncl) {
+        const float* pr = cluster.map_shared_rank(part_s, lane) + i * kPartStride;
+        Mk = pr[16];
+        lk = pr[17];
+      }
+      float M = lk > 0.f ? Mk : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float wk = (lk > 0.f) ? sm100::ex2_approx(Mk - M) : 0.f;
+      float den = wk * lk;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      // lane c (< 16) sums column c over the parts
+      float num = 0.f;
+      for (int k = 0; k < a.ncl; ++k) {
+        const float w_k = __shfl_sync(0xffffffffu, wk, k);
+        if (lane < D16 && w_k > 0.f) num = fmaf(w_k, cluster.map_shared_rank(part_s, k)[i * kPartStride + lane], num);
+      }
+      const float val = den > 0.f ? num / den : 0.f;
+      const float nb = __shfl_down_sync(0xffffffffu, val, 1);
+      if (lane < D16 && (lane & 1) == 0) {
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + o_off(p, b, h, i);
+        *reinterpret_cast<uint32_t*>(orow + lane) = pack2(val, nb);
+      }
+      if (lane == 0 && p.lse) p.lse[zq * p.Tq + i] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
+    }
+  }
+  // keep every part's shared memory alive until CTA 0 has read it
+  cluster.sync();
+}
+
 }  // namespace
 
 int small_d_check(const Params& p, sdpa_dtype_t dtype) {
@@ -419,6 +602,34 @@ cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream
 }
 
 cudaError_t launch_split_kv(const Params& p, cudaStream_t stream) {
+  // one cluster of up to 8 parts per (batch, head) when the key axis fits
+  if (p.Tq <= kRowsMax && p.Tkv >= 1 && p.Tkv <= (long long)kClusterMax * kClusterChunk && p.B <= 65535 &&
+      p.Hq <= 65535) {
+    ClusterArgs a;
+    a.p = p;
+    a.ncl = kClusterMax;
+    a.chunk = (p.Tkv + kClusterMax - 1) / kClusterMax;
+    const size_t smem = (size_t)2 * kClusterChunk * (D16 / 4) * sizeof(float4) + (size_t)kRowsMax * kPartStride * 4;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [&] {
+      attr = cudaFuncSetAttribute(split_kv_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    if (attr != cudaSuccess) return attr;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.ncl, (unsigned)p.Hq, (unsigned)p.B);
+    cfg.blockDim = dim3(kSplitThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)a.ncl;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, split_kv_cluster_kernel, a);
+  }
   size_t cb = 0, db = 0;
   split_kv_workspace_bytes(p, &cb, &db);
   void *cnt = nullptr, *data = nullptr;
