@@ -20,6 +20,9 @@
 //    chunk (lanes stride the keys), and writes (m, l, unnormalised O) for its
 //    part.  The last CTA of a (batch, head) to finish, detected with an
 //    atomic ticket, merges the parts: O = sum_k 2^(m_k-M) O_k / sum_k 2^(m_k-M) l_k.
+//    When the key axis fits in 8 parts, split_kv_cluster_kernel does the
+//    same with the parts in one thread-block cluster, merged through
+//    distributed shared memory instead of a global workspace.
 //
 // Both take every mask kind and GQA; neither takes the rel-pos bias (the
 // exact kernel does).

@@ -138,10 +138,12 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_
  *          sum-exp of each score row (m + log l; -inf for a row with no
  *          visible key).
  *   path : sdpa_path_t; AUTO behaves like sdpa_fwd.
- * The split-KV path keeps its partial results in a scratch buffer that the
- * library allocates on first use per device and grows when needed (never
- * freed until exit); calls on one device that overlap on the GPU must not use
- * that path concurrently.
+ * The split-KV path merges its parts inside a thread-block cluster when the
+ * key axis fits in 8 parts of 512 keys and there are at most 64 query rows;
+ * otherwise -- and the tensor-core path when it splits a key range -- it
+ * keeps partial results in a scratch buffer that the library allocates on
+ * first use per device and grows when needed (never freed until exit); calls
+ * on one device that overlap on the GPU must not use such a path concurrently.
  */
 int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
                 int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
