@@ -18,9 +18,9 @@ LIB_PATH = os.path.join(_PKG, "libsdpa.so")
 
 SDPA_F32, SDPA_BF16 = 0, 1
 MASK_NONE, MASK_CAUSAL, MASK_SLIDING, MASK_FLOAT, MASK_BOOL = 0, 1, 2, 3, 4
-PATH_AUTO, PATH_EXACT, PATH_TCGEN05, PATH_SMALL_D, PATH_SPLIT_KV = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_EXACT, PATH_TCGEN05, PATH_SMALL_D, PATH_SPLIT_KV, PATH_TC_PERSISTENT = 0, 1, 2, 3, 4, 5
 PATHS = {"auto": PATH_AUTO, "exact": PATH_EXACT, "tcgen05": PATH_TCGEN05,
-         "small_d": PATH_SMALL_D, "split_kv": PATH_SPLIT_KV}
+         "small_d": PATH_SMALL_D, "split_kv": PATH_SPLIT_KV, "tc_persistent": PATH_TC_PERSISTENT}
 STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
           -3: "SDPA_ERR_MISALIGNED", -4: "SDPA_ERR_CUDA", -5: "SDPA_ERR_TIMEOUT",
           -6: "SDPA_ERR_CAPACITY"}

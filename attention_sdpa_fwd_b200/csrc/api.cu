@@ -169,7 +169,11 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
 int choose_path(const Problem& pr) {
   const Params& p = pr.p;
   if (p.Tkv == 0) return SDPA_PATH_EXACT;
-  if (tc_check(p, pr.dtype) == SDPA_OK) return SDPA_PATH_TCGEN05;
+  if (tc_check(p, pr.dtype) == SDPA_OK) {
+    // many short problems: one persistent CTA per SM walks them
+    if (tc_persist_check(p, pr.dtype) == SDPA_OK && tc_persist_preferred(p)) return SDPA_PATH_TC_PERSISTENT;
+    return SDPA_PATH_TCGEN05;
+  }
   if (small_d_check(p, pr.dtype) == SDPA_OK) {
     // few query rows against a long key axis: split the keys over the SMs
     if (p.Tq <= 64 && p.Tkv >= 1024) return SDPA_PATH_SPLIT_KV;
@@ -191,6 +195,12 @@ int run(const Problem& pr, int path, cudaStream_t stream) {
       const int rc = tc_check(p, pr.dtype);
       if (rc != SDPA_OK) return rc;
       e = launch_tc(p, stream);
+      break;
+    }
+    case SDPA_PATH_TC_PERSISTENT: {
+      const int rc = tc_persist_check(p, pr.dtype);
+      if (rc != SDPA_OK) return rc;
+      e = launch_tc_persist(p, stream);
       break;
     }
     case SDPA_PATH_SMALL_D: {
@@ -275,7 +285,7 @@ extern "C" int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* ou
                            int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
                            const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
                            const int* q_hw, const int* k_hw, float* lse, int path, cudaStream_t stream) {
-  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_SPLIT_KV) return SDPA_ERR_INVALID_ARG;
+  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_TC_PERSISTENT) return SDPA_ERR_INVALID_ARG;
   Problem pr;
   int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
                          rel_pos_h, rel_pos_w, q_hw, k_hw, lse, &pr);
@@ -289,7 +299,7 @@ extern "C" int sdpa_fwd_strided(const void* q, const sdpa_strides_t* q_strides, 
                                 int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind, const void* mask_ptr,
                                 const void* rel_pos_h, const void* rel_pos_w, const int* q_hw, const int* k_hw,
                                 float* lse, int path, cudaStream_t stream) {
-  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_SPLIT_KV) return SDPA_ERR_INVALID_ARG;
+  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_TC_PERSISTENT) return SDPA_ERR_INVALID_ARG;
   const sdpa_strides_t* st[4] = {q_strides, k_strides, v_strides, out_strides};
   Problem pr;
   int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
@@ -369,7 +379,7 @@ extern "C" int sdpa_fwd_host(const void* q, const void* k, const void* v, void* 
                              int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int mask_kind,
                              const void* mask_ptr, const void* rel_pos_h, const void* rel_pos_w,
                              const int* q_hw, const int* k_hw, int path, cudaStream_t stream) {
-  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_SPLIT_KV) return SDPA_ERR_INVALID_ARG;
+  if (path < SDPA_PATH_AUTO || path > SDPA_PATH_TC_PERSISTENT) return SDPA_ERR_INVALID_ARG;
   Problem pr;
   int rc = build_problem(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale, mask_kind, mask_ptr,
                          rel_pos_h, rel_pos_w, q_hw, k_hw, nullptr, &pr);

@@ -101,6 +101,10 @@ cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream
 int split_kv_static(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
 int num_sms();
 cudaError_t launch_tc(const Params& p, cudaStream_t stream);
+// persistent form of the tensor-core kernel (one CTA per SM over many short problems)
+int tc_persist_check(const Params& p, sdpa_dtype_t dtype);
+bool tc_persist_preferred(const Params& p);
+cudaError_t launch_tc_persist(const Params& p, cudaStream_t stream);
 
 // Parts sdpa_merge combines at most.
 constexpr int kMaxMergeParts = 16;

@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   tc_fence_after();
   const uint32_t tbase = *tslot;
   volatile int* abort_v = abort_flag;
-  constexpr bool kWarpIssue = !kPSep;
+  constexpr bool kWarpIssue = true;
   auto mma_ss_x = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
     if constexpr (kWarpIssue) mma_ss_w(d, a, b, id, acc); else mma_ss(d, a, b, id, acc);
   };
@@ -342,8 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // At head_dim 128 the whole warp runs the loop and one elected lane issues
-    // each instruction (measured faster there); at 64 lane 0 runs it alone.
+    // The whole warp runs the loop (every wait is warp-uniform) and one elected
+    // lane issues each instruction: measured faster than lane 0 running it
+    // alone (SAM global attention, head_dim 64: 100.4 against 110.8 us).
     if ((kWarpIssue || lane == 0) && n_tiles > 0) {
       constexpr uint32_t id_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t id_pv = idesc_bf16_f32(128, D, false, true);

@@ -64,6 +64,25 @@ def test_valid_problem_selects_a_path(L):
     assert sel() >= 0
 
 
+def test_auto_takes_persistent_form_for_many_short_problems(L):
+    """SAM windowed attention (100 windows x 12 heads of 14x14 tokens), with or
+    without the rel-pos bias, takes the persistent tensor-core form; SAM global
+    attention (one 64x64 grid, 12 heads: 16 query blocks per head), masked
+    problems and long key axes keep the one-CTA-per-block form."""
+    rh, rw = 0x500000, 0x600000
+    far = dict(q=0x10000000, k=0x20000000, v=0x30000000, out=0x40000000)  # spans of up to 256 MB apart
+    sel_far = lambda **kw: sel(**far, **kw)
+    win = dict(B=100, Hq=12, Hkv=12, Tq=196, Tkv=196, rh=rh, rw=rw, q_hw=(ctypes.c_int * 2)(14, 14),
+               k_hw=(ctypes.c_int * 2)(14, 14))
+    assert sel_far(**win) == S.PATH_TC_PERSISTENT
+    glob = dict(B=1, Hq=12, Hkv=12, Tq=4096, Tkv=4096, rh=rh, rw=rw, q_hw=(ctypes.c_int * 2)(64, 64),
+                k_hw=(ctypes.c_int * 2)(64, 64))
+    assert sel_far(**glob) == S.PATH_TCGEN05
+    assert sel_far(B=100, Hq=12, Hkv=12, Tq=196, Tkv=196, mask_kind=S.MASK_CAUSAL) == S.PATH_TCGEN05
+    assert sel_far(B=100, Hq=12, Hkv=12, Tq=196, Tkv=196) == S.PATH_TC_PERSISTENT
+    assert sel_far(B=100, Hq=12, Hkv=12, Tq=196, Tkv=700) == S.PATH_TCGEN05   # > 4 key tiles per block
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(Hq=3, Hkv=2), -1),                 # Hq % Hkv != 0
     (dict(Hkv=0), -1),

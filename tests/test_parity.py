@@ -89,10 +89,23 @@ CASES = [
        mask_neg_inf_frac=0.2, mask_heads=1, seed=36),
     S_("float_bf16_d128_odd_tiles", BF16, 2, 3, 3, 200, 300, 128, mask_kind=W.MASK_FLOAT, mask_std=2.0,
        mask_neg_inf_frac=0.1, mask_heads=3, seed=37),
+    # more query blocks than SMs: the persistent form walks several per CTA
+    # (consecutive units of one CTA differ in window, head and query block)
+    S_("persist_relpos_14x14_many", BF16, 40, 4, 4, 196, 196, 64, q_hw=(14, 14), k_hw=(14, 14), rel_std=0.5,
+       seed=50),
+    S_("persist_relpos_16x16_many", BF16, 20, 8, 8, 256, 256, 64, q_hw=(16, 16), k_hw=(16, 16), rel_std=0.5,
+       seed=51),
+    S_("persist_relpos_6x14_many", BF16, 50, 4, 2, 84, 84, 64, q_hw=(6, 14), k_hw=(6, 14), rel_std=1.0, seed=52),
+    S_("persist_none_ragged_many", BF16, 8, 12, 3, 260, 300, 64, seed=53),
+    S_("persist_none_four_tiles_many", BF16, 10, 16, 16, 100, 500, 64, seed=54),
+    # three or four units per CTA: both Q buffers are refilled after their
+    # first unit (the hand-over that waits for the unit two back)
+    S_("persist_relpos_14x14_deep", BF16, 80, 6, 6, 196, 196, 64, q_hw=(14, 14), k_hw=(14, 14), rel_std=0.5,
+       seed=55),
 ]
 CASE_IDS = [c.name for c in CASES]
 
-PATHS = ["exact", "tcgen05", "small_d", "split_kv"]
+PATHS = ["exact", "tcgen05", "small_d", "split_kv", "tc_persistent"]
 
 
 def applicable(path: str, sp: W.Spec) -> bool:
@@ -113,6 +126,10 @@ def applicable(path: str, sp: W.Spec) -> bool:
         return True
     if path in ("small_d", "split_kv"):
         return sp.d == 16 and not sp.rel
+    if path == "tc_persistent":
+        if sp.d != 64 or sp.mask_kind != W.MASK_NONE:
+            return False
+        return (not sp.rel) or (sp.k_hw[1] in (14, 16) and sp.k_hw[0] <= 16)
     return False
 
 
@@ -121,7 +138,7 @@ def _implemented(path):
     return path in _BUILT
 
 
-_BUILT = {"exact", "tcgen05", "small_d", "split_kv"}
+_BUILT = {"exact", "tcgen05", "small_d", "split_kv", "tc_persistent"}
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -184,6 +201,21 @@ def _edge_cases(path):
     torch.cuda.synchronize()
     assert torch.all(o2[0, 0, 3] == 0) and torch.all(o2[0, 0, 129] == 0)
     assert torch.all(o2[0, 0, 4].abs().sum() > 0)
+
+
+def test_persistent_edges():
+    """Persistent form: a single key, a single query, B = 0, and more SMs than units."""
+    import attention_sdpa_fwd_b200 as S
+    dev = "cuda"
+    q1 = torch.randn(3, 2, 1, 64, device=dev, dtype=BF16)
+    k1 = torch.randn(3, 2, 1, 64, device=dev, dtype=BF16)
+    v1 = torch.randn(3, 2, 1, 64, device=dev, dtype=BF16)
+    o1 = S.sdpa(q1, k1, v1, path="tc_persistent")
+    torch.cuda.synchronize()
+    assert torch.equal(o1, v1)
+    z = torch.empty(0, 2, 5, 64, device=dev, dtype=BF16)
+    S.sdpa(z, z, z, 0.1, path="tc_persistent")
+    torch.cuda.synchronize()
 
 
 def test_host_entry_point_matches_device_entry_point():
