@@ -185,37 +185,27 @@ int choose_path(const Problem& pr) {
 int run(const Problem& pr, int path, cudaStream_t stream) {
   if (pr.empty_out) return SDPA_OK;
   Params p = pr.p;
+  if (path == SDPA_PATH_AUTO) path = choose_path(pr);
+  // a forced family that cannot take the problem says so before any device work
+  int rc = SDPA_OK;
+  switch (path) {
+    case SDPA_PATH_EXACT: break;
+    case SDPA_PATH_TCGEN05: rc = tc_check(p, pr.dtype); break;
+    case SDPA_PATH_TC_PERSISTENT: rc = tc_persist_check(p, pr.dtype); break;
+    case SDPA_PATH_SMALL_D: rc = small_d_check(p, pr.dtype); break;
+    case SDPA_PATH_SPLIT_KV: rc = split_kv_check(p, pr.dtype); break;
+    default: return SDPA_ERR_INVALID_ARG;
+  }
+  if (rc != SDPA_OK) return rc;
   p.err = error_word_ptr();
   if (p.err == nullptr) return SDPA_ERR_CUDA;
-  if (path == SDPA_PATH_AUTO) path = choose_path(pr);
-  cudaError_t e;
+  cudaError_t e = cudaErrorInvalidValue;
   switch (path) {
     case SDPA_PATH_EXACT: e = launch_exact(p, pr.dtype, stream); break;
-    case SDPA_PATH_TCGEN05: {
-      const int rc = tc_check(p, pr.dtype);
-      if (rc != SDPA_OK) return rc;
-      e = launch_tc(p, stream);
-      break;
-    }
-    case SDPA_PATH_TC_PERSISTENT: {
-      const int rc = tc_persist_check(p, pr.dtype);
-      if (rc != SDPA_OK) return rc;
-      e = launch_tc_persist(p, stream);
-      break;
-    }
-    case SDPA_PATH_SMALL_D: {
-      const int rc = small_d_check(p, pr.dtype);
-      if (rc != SDPA_OK) return rc;
-      e = launch_small_d(p, stream);
-      break;
-    }
-    case SDPA_PATH_SPLIT_KV: {
-      const int rc = split_kv_check(p, pr.dtype);
-      if (rc != SDPA_OK) return rc;
-      e = launch_split_kv(p, stream);
-      break;
-    }
-    default: return SDPA_ERR_INVALID_ARG;
+    case SDPA_PATH_TCGEN05: e = launch_tc(p, stream); break;
+    case SDPA_PATH_TC_PERSISTENT: e = launch_tc_persist(p, stream); break;
+    case SDPA_PATH_SMALL_D: e = launch_small_d(p, stream); break;
+    case SDPA_PATH_SPLIT_KV: e = launch_split_kv(p, stream); break;
   }
   return e == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
 }

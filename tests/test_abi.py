@@ -133,6 +133,38 @@ def test_forward_rejects_before_launch(L):
     assert rc == -2
 
 
+def fwd_ex(path, **kw):
+    args = dict(q=Q, k=K, v=V, out=O, dtype=BF16, B=1, Hq=4, Hkv=2, Tq=8, Tkv=8, d=64,
+                mask_kind=0, mask=None, rh=None, rw=None, q_hw=None, k_hw=None)
+    args.update(kw)
+    m = args["mask"]
+    return S.sdpa_fwd_ex(args["q"], args["k"], args["v"], args["out"], args["dtype"], args["B"], args["Hq"],
+                         args["Hkv"], args["Tq"], args["Tkv"], args["d"], 0.125, args["mask_kind"],
+                         ctypes.byref(m) if m is not None else None, args["rh"], args["rw"], args["q_hw"],
+                         args["k_hw"], None, path, None)
+
+
+REL14 = dict(rh=0x600000, rw=0x700000, Tq=196, Tkv=196, q_hw=(14, 14), k_hw=(14, 14))
+
+
+@pytest.mark.parametrize("path,kw", [
+    (S.PATH_TC_PERSISTENT, dict(d=128)),                                   # head_dim 64 only
+    (S.PATH_TC_PERSISTENT, dict(d=16)),
+    (S.PATH_TC_PERSISTENT, dict(dtype=S.SDPA_F32)),                         # bf16 only
+    (S.PATH_TC_PERSISTENT, dict(mask_kind=S.MASK_CAUSAL, mask=S.sdpa_mask_t())),
+    (S.PATH_TC_PERSISTENT, dict(REL14, q_hw=(7, 28), k_hw=(7, 28))),          # key-grid width 28
+    (S.PATH_TC_PERSISTENT, dict(REL14, Tq=238, Tkv=238, q_hw=(17, 14), k_hw=(17, 14))),  # height 17 > 16
+    (S.PATH_TCGEN05, dict(d=16)),
+    (S.PATH_TCGEN05, dict(REL14, q_hw=(7, 28), k_hw=(7, 28))),
+    (S.PATH_SMALL_D, dict(d=64)),
+    (S.PATH_SPLIT_KV, dict(REL14, d=16)),
+])
+def test_forced_path_rejected_before_launch(L, path, kw):
+    """A forced kernel family that cannot take the problem returns
+    SDPA_ERR_UNSUPPORTED before any device work (no GPU needed)."""
+    assert fwd_ex(path, **kw) == -2
+
+
 def test_binding_has_no_cpu_path():
     import torch
     q = torch.zeros(1, 1, 4, 16)
