@@ -230,6 +230,30 @@ def launch(S, spec: W.Spec, st, stream, path):
         raise RuntimeError(f"sdpa_fwd_ex failed: {S.STATUS.get(rc, rc)}")
 
 
+def auto_path_name(S, spec: W.Spec) -> str:
+    """The kernel family AUTO dispatches this workload to (host-side query: the
+    library validates but never dereferences the placeholder addresses, which
+    are 2^40 bytes apart so that no two spans overlap)."""
+    import ctypes
+    base = 1 << 40
+    data = base * 7 if spec.mask_kind in (W.MASK_FLOAT, W.MASK_BOOL) else None
+    m = None
+    if spec.mask_kind != W.MASK_NONE:
+        m = S.sdpa_mask_t(offset=spec.offset, window=spec.window, data=data)
+        if data is not None:  # strides of the workload's contiguous [B, mask_heads, Tq, Tkv] mask
+            m.stride_b = 0 if spec.B == 1 else spec.mask_heads * spec.Tq * spec.Tkv
+            m.stride_h = 0 if spec.mask_heads == 1 else spec.Tq * spec.Tkv
+            m.stride_q = spec.Tkv
+    rel = spec.q_hw is not None
+    rc = S.sdpa_select_path(base, base * 2, base * 3, base * 4,
+                            S.SDPA_BF16 if spec.dtype == torch.bfloat16 else S.SDPA_F32,
+                            spec.B, spec.Hq, spec.Hkv, spec.Tq, spec.Tkv, spec.d, spec.mask_kind,
+                            ctypes.byref(m) if m is not None else None,
+                            base * 5 if rel else None, base * 6 if rel else None, spec.q_hw, spec.k_hw)
+    names = {v: k for k, v in S.PATHS.items()}
+    return names.get(rc, f"status {rc}")
+
+
 def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, ws: int, path=0):
     per_set = spec.bytes()
     nsets = max(2, math.ceil(2 * L2_BYTES / max(per_set, 1)))
@@ -446,7 +470,8 @@ def run_ours(args):
             gm = time_graph(S, sp, device)
             hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
             bf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-            per_config[name] = dict(ms=lm, graph_ms=gm, tflops=sp.flops() / (gm * 1e-3) / 1e12,
+            per_config[name] = dict(path=auto_path_name(S, sp), ms=lm, graph_ms=gm,
+                                    tflops=sp.flops() / (gm * 1e-3) / 1e12,
                                     gbs=sp.bytes() / (gm * 1e-3) / 1e9,
                                     frac_bf16=sp.flops() / (gm * 1e-3) / 1e12 / bf,
                                     frac_hbm=sp.bytes() / (gm * 1e-3) / 1e9 / hbm)
