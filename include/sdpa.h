@@ -142,7 +142,10 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_
  *   lse  : NULL, or a device float [B, Hq, Tq] receiving the natural-log
  *          sum-exp of each score row (m + log l; -inf for a row with no
  *          visible key).
- *   path : sdpa_path_t; AUTO behaves like sdpa_fwd.
+ *   path : sdpa_path_t; AUTO behaves like sdpa_fwd.  A forced family that
+ *          cannot take the problem returns SDPA_ERR_UNSUPPORTED (or
+ *          SDPA_ERR_MISALIGNED) before any device work.
+ * The persistent tensor-core path allocates nothing and writes no scratch.
  * The split-KV path merges its parts inside a thread-block cluster when the
  * key axis fits in 8 parts of 512 keys and there are at most 64 query rows;
  * otherwise -- and the tensor-core path when it splits a key range -- it
