@@ -157,7 +157,16 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
     const size_t nk = span(p.skb, p.skh, p.skt, Hkv, Tkv), nv = span(p.svb, p.svh, p.svt, Hkv, Tkv);
     if (overlaps(out, no, q, nq) || overlaps(out, no, k, nk) || overlaps(out, no, v, nv))
       return SDPA_ERR_INVALID_ARG;
-    if (lse && (overlaps(lse, (size_t)rows * 4, out, no) || overlaps(lse, (size_t)rows * 4, q, nq)))
+    // lse is written while other CTAs still read q, k, v and the mask: no overlap with any of them
+    size_t nm = 0;
+    if (p.mask != nullptr && Tkv > 0) {
+      const long long last = (long long)(B - 1) * p.msb + (long long)(Hq - 1) * p.msh +
+                             (long long)(Tq - 1) * p.msq + Tkv;
+      nm = (size_t)last * (mask_kind == SDPA_MASK_BOOL ? 1 : esz);
+    }
+    const size_t nl = (size_t)rows * 4;
+    if (lse && (overlaps(lse, nl, out, no) || overlaps(lse, nl, q, nq) || overlaps(lse, nl, k, nk) ||
+                overlaps(lse, nl, v, nv) || overlaps(lse, nl, p.mask, nm)))
       return SDPA_ERR_INVALID_ARG;
   }
   p.k_vec16 = (k != nullptr && aligned(k, 16) && (p.skb * (long long)esz) % 16 == 0 &&

@@ -12,6 +12,8 @@
 // Every call on a device shares it, and each call leaves its contents behind,
 // so two calls whose kernels overlap on the GPU (different streams, or no
 // ordering between them) race on it; calls on one stream are fine.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace sdpa {
@@ -26,13 +28,17 @@ __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDev = 64;
 
-// The array's device address, looked up once per device.  Host code must not
-// use the symbol itself: on the host it names a host-side stand-in, and a
-// kernel given that address would fault (or quietly read the wrong memory).
+// The array's device address, looked up once per device (under a lock, so
+// that two host threads making their first call on one device at once do not
+// race on the cache).  Host code must not use the symbol itself: on the host
+// it names a host-side stand-in, and a kernel given that address would fault
+// (or quietly read the wrong memory).
 int static_scratch(void** ptr) {
   static void* addr[kMaxDev] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return SDPA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SDPA_ERR_CUDA;

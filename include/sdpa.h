@@ -152,6 +152,11 @@ int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_
  * keeps partial results in a scratch buffer that the library allocates on
  * first use per device and grows when needed (never freed until exit); calls
  * on one device that overlap on the GPU must not use such a path concurrently.
+ * Growing that buffer is the one place an otherwise asynchronous call blocks
+ * the host: before it frees the smaller buffer it calls
+ * cudaDeviceSynchronize(), because earlier launches may still be using it.
+ * A caller that wants no such stall makes one call at its largest size first.
+ * lse must not overlap q, k, v, out or the mask tensor (SDPA_ERR_INVALID_ARG).
  */
 int sdpa_fwd_ex(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
                 int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
@@ -259,6 +264,8 @@ int sdpa_fwd_host(const void* q, const void* k, const void* v, void* out, sdpa_d
  * shares the array and leaves its contents behind: calls whose kernels may
  * overlap on the GPU (different streams without ordering between them) race
  * on it and must not be issued; calls on one stream are ordered and safe.
+ * Such a race is not detected: it gives wrong output silently, not an error
+ * status from sdpa_last_device_error.
  */
 int sdpa_fwd_split_kv_static(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
                              int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,

@@ -203,3 +203,17 @@ def test_merge_validates_on_host(L):
     assert S.sdpa_merge(o, l, 2, (1 << 20) + 8, 1 << 21, **ok) == -3     # out not 16-byte aligned
     assert S.sdpa_merge(o, l, 2, 8192 + 64, 1 << 21, **ok) == -1         # out overlaps part 1
     assert S.sdpa_merge(o, l, 2, 1 << 20, None, **dict(ok, Tq=0)) == 0   # nothing to do
+
+
+@pytest.mark.parametrize("where", ["q", "k", "v", "out", "mask"])
+def test_lse_overlapping_an_input_is_rejected(L, where):
+    """lse is written while other CTAs still read q, k, v and the mask tensor:
+    an lse buffer that overlaps any of them (or out) is an argument error,
+    reported before any launch."""
+    mask_data = 0x500000
+    m = S.sdpa_mask_t(data=mask_data, stride_b=0, stride_h=0, stride_q=8)
+    at = dict(q=Q, k=K, v=V, out=O, mask=mask_data)[where]
+    lse = ctypes.c_void_p(at + 4)
+    rc = S.sdpa_fwd_ex(Q, K, V, O, BF16, 1, 4, 2, 8, 8, 64, 0.125, S.MASK_FLOAT, ctypes.byref(m),
+                       None, None, None, None, lse, 0, None)
+    assert rc == -1

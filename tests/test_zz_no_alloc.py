@@ -12,7 +12,8 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import GATES, stats
+import oracle
+from helpers import GATES, assert_gates, stats
 
 pytestmark = pytest.mark.gpu
 
@@ -34,20 +35,28 @@ def _static_call(S, q, k, v, out, lse, scale, mask_kind=0, mask=None):
                                       torch.cuda.current_stream().cuda_stream)
 
 
-def test_static_scratch_entry_matches_split_kv_twice():
+def test_static_scratch_entry_matches_split_kv_and_oracle_twice():
+    """Two calls in a row (the second reuses the scratch the first one left
+    behind): each agrees with the regular split-KV entry point and with the
+    fp64 oracle, within the bf16 gates; lse within 2e-3 of the oracle's."""
     import attention_sdpa_fwd_b200 as S
     q, k, v = _inputs(4, 8, 8, 4096, seed=11)
     ref_lse = torch.empty(4, 8, 8, device="cuda")
     ref = S.sdpa(q, k, v, 0.25, lse=ref_lse, path="split_kv")
-    for call in range(2):  # the second call reuses the scratch the first one left behind
+    torch.cuda.synchronize()
+    orc = oracle.sdpa(q.cpu(), k.cpu(), v.cpu(), 0.25)
+    for call in range(2):
         out = torch.full_like(q, float("nan"))
         lse = torch.empty_like(ref_lse)
         assert _static_call(S, q, k, v, out, lse, 0.25) == 0
         torch.cuda.synchronize()
         assert S.sdpa_last_device_error(torch.cuda.current_stream().cuda_stream) == 0
-        s = stats(out.double().cpu().numpy(), ref.double().cpu().numpy())
+        got = out.double().cpu().numpy()
+        s = stats(got, ref.double().cpu().numpy())
         assert all(s[key] <= GATES[torch.bfloat16][key] for key in GATES[torch.bfloat16]), (call, s)
         assert torch.allclose(lse, ref_lse, atol=1e-3, rtol=0), call
+        assert_gates(got, orc.out, torch.bfloat16, f"static entry vs oracle, call {call}")
+        assert np.max(np.abs(lse.double().cpu().numpy() - orc.lse)) < 2e-3, call
 
 
 def test_static_scratch_entry_with_mask_and_a_new_shape():
@@ -59,8 +68,11 @@ def test_static_scratch_entry_with_mask_and_a_new_shape():
     out = torch.empty_like(q)
     assert _static_call(S, q, k, v, out, None, 0.25, S.MASK_BOOL, keep) == 0
     torch.cuda.synchronize()
-    s = stats(out.double().cpu().numpy(), ref.double().cpu().numpy())
+    got = out.double().cpu().numpy()
+    s = stats(got, ref.double().cpu().numpy())
     assert all(s[key] <= GATES[torch.bfloat16][key] for key in GATES[torch.bfloat16]), s
+    orc = oracle.sdpa(q.cpu(), k.cpu(), v.cpu(), 0.25, mask_kind=S.MASK_BOOL, mask=keep.cpu())
+    assert_gates(got, orc.out, torch.bfloat16, "static entry with a bool mask vs oracle")
 
 
 def test_static_scratch_entry_rejects_oversized_problems():
