@@ -98,7 +98,10 @@ def sdpa(q, k, v, scale: float, *, mask_kind: int = MASK_NONE, offset: int = 0,
 
     q [B,Hq,Tq,d]; k, v [B,Hkv,Tkv,d]; ``mask`` is a float (MASK_FLOAT) or
     boolean/uint8 (MASK_BOOL) array broadcastable to [B,Hq,Tq,Tkv] (size-1
-    axes broadcast); rel_pos_h [2*k_hw[0]-1, d] and rel_pos_w [2*k_hw[1]-1, d].
+    axes broadcast); rel_pos_h [q_hw[0]+k_hw[0]-1, d] and rel_pos_w
+    [q_hw[1]+k_hw[1]-1, d] (2*K-1 rows each when the query and key grids are
+    equal; with grids of their own, the offset qh - kh runs over
+    -(Kh-1) .. Qh-1 and the shift Kh-1 maps it onto the table's rows).
     ``rows`` restricts the computation to those query rows (same rows for
     every (b, h)); the result then has len(rows) rows."""
     lib = lib or load()
@@ -127,6 +130,9 @@ def sdpa(q, k, v, scale: float, *, mask_kind: int = MASK_NONE, offset: int = 0,
     rh, rw = _f64(rel_pos_h), _f64(rel_pos_w)
     qh, qw = (q_hw if q_hw is not None else (0, 0))
     kh, kw = (k_hw if k_hw is not None else (0, 0))
+    if rh is not None and rw is not None:
+        if rh.shape != (qh + kh - 1, d) or rw.shape != (qw + kw - 1, d):
+            raise ValueError("rel tables must be [q_hw[0]+k_hw[0]-1, d] and [q_hw[1]+k_hw[1]-1, d]")
     rows_arr = None
     n = Tq
     if rows is not None:

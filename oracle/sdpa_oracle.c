@@ -31,6 +31,12 @@
  *   rel_w[i, kw] = sum_c q[i,c] * Rw[qw(i) - kw + Kw - 1, c]
  *   qh(i) = i / Qw, qw(i) = i % Qw, kh(j) = j / Kw, kw(j) = j % Kw
  *
+ * (Qh, Qw) is the query patch grid and (Kh, Kw) the key patch grid.  They may
+ * differ: the formula is read with each coordinate taken from its own grid
+ * and the shift from the key grid, so the offset qh - kh runs from -(Kh - 1)
+ * to Qh - 1 and Rh needs Qh + Kh - 1 rows (Rw: Qw + Kw - 1); with equal grids
+ * that is the 2*K - 1 rows of SAM's tables.
+ *
  * Readings of what the pages leave open (each one stated where it is used):
  *   - GQA/MQA "repeat key/value heads to match the query": each kv head is
  *     repeated g = Hq/Hkv times consecutively, so hk = h / g.
@@ -92,7 +98,7 @@ static double dot(const double* a, const double* b, int n) {
  *   out [B, Hq,  nrows, d]    lse  [B, Hq, nrows]      (lse may be NULL)
  *   weights [B, Hq, nrows, Tkv] (may be NULL; the softmax weights p/l)
  *   fmask / bmask: element (b, h, i, j) at b*msb + h*msh + i*msq + j
- *   rel_h [2*k_h - 1, d], rel_w [2*k_w - 1, d]  (both NULL: no rel-pos term)
+ *   rel_h [q_h + k_h - 1, d], rel_w [q_w + k_w - 1, d]  (both NULL: no rel-pos term)
  * Returns 0, or -1 on an inconsistent argument.
  */
 int oracle_sdpa_rows(const double* q, const double* k, const double* v,
@@ -153,6 +159,8 @@ int oracle_sdpa_rows(const double* q, const double* k, const double* v,
         for (int a = 0; a < k_h; ++a) {
 #if ORACLE_PLANT == 1
           const long long idx = a - qh + k_h - 1;
+#elif ORACLE_PLANT == 13
+          const long long idx = (qh - a + q_h - 1 + (q_h + k_h - 1)) % (q_h + k_h - 1);
 #else
           const long long idx = qh - a + k_h - 1;
 #endif
@@ -163,7 +171,11 @@ int oracle_sdpa_rows(const double* q, const double* k, const double* v,
 #endif
         }
         for (int a = 0; a < k_w; ++a) {
+#if ORACLE_PLANT == 13
+          const long long idx = (qw - a + q_w - 1 + (q_w + k_w - 1)) % (q_w + k_w - 1);
+#else
           const long long idx = qw - a + k_w - 1;
+#endif
 #if ORACLE_PLANT == 2
           relw[a] = 0.0;
 #else

@@ -27,8 +27,12 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 def _num(x):
     if isinstance(x, str):
         table = {"ln2": math.log(2.0), "ln3": math.log(3.0), "ln4": math.log(4.0),
-                 "-ln2": -math.log(2.0), "2ln3": 2.0 * math.log(3.0), "-inf": -math.inf}
-        return table[x]
+                 "-ln2": -math.log(2.0), "2ln3": 2.0 * math.log(3.0), "-inf": -math.inf,
+                 "ln(9/2)": math.log(4.5), "ln(7/2)": math.log(3.5)}
+        if x in table:
+            return table[x]
+        num, den = x.split("/")  # an exact fraction "a/b"
+        return float(num) / float(den)
     if isinstance(x, list):
         return [_num(y) for y in x]
     return float(x)
@@ -69,6 +73,16 @@ def _rand_problem(seed, B=1, Hq=2, Hkv=1, Tq=6, Tkv=6, d=4, hw=(2, 3), rel=True,
 def _bias_from_index_table(q, Rh, Rw):
     """Bias [B,H,6,6] of the 2x3 grid from the hand-enumerated index table."""
     rows = np.loadtxt(os.path.join(GOLDEN, "relpos_index_2x3.txt"), dtype=np.int64, comments="#")
+    bias = np.zeros(q.shape[:2] + (6, 6))
+    for i, j, ih, iw in rows:
+        bias[:, :, i, j] = q[:, :, i, :] @ Rh[ih] + q[:, :, i, :] @ Rw[iw]
+    return bias
+
+
+def _bias_from_index_table_q2x3_k3x2(q, Rh, Rw):
+    """Bias [B,H,6,6] of query grid 2x3 against key grid 3x2 from the
+    hand-enumerated index table."""
+    rows = np.loadtxt(os.path.join(GOLDEN, "relpos_index_q2x3_k3x2.txt"), dtype=np.int64, comments="#")
     bias = np.zeros(q.shape[:2] + (6, 6))
     for i, j, ih, iw in rows:
         bias[:, :, i, j] = q[:, :, i, :] @ Rh[ih] + q[:, :, i, :] @ Rw[iw]
@@ -173,6 +187,43 @@ def pin_index_table_2x3(lib):
         torch.from_numpy(p["q"]), torch.from_numpy(p["k"]), torch.from_numpy(p["v"]),
         attn_mask=torch.from_numpy(bias), scale=0.45)
     _close(r.out, t.numpy(), 1e-12, "2x3 index table")
+
+
+def pin_index_table_q2x3_k3x2(lib):
+    """Query and key grids of their own (2x3 against 3x2): the rel-pos bias
+    matches the hand-enumerated index table, through torch's float64 SDPA
+    given the bias as its additive mask."""
+    r = _rng(16)
+    q, k, v = (r.standard_normal((1, 2, 6, 3)) for _ in range(3))
+    Rh = r.standard_normal((4, 3)) * 0.8
+    Rw = r.standard_normal((4, 3)) * 0.8
+    bias = _bias_from_index_table_q2x3_k3x2(q, Rh, Rw)
+    res = oracle.sdpa(q, k, v, 0.45, rel_pos_h=Rh, rel_pos_w=Rw, q_hw=(2, 3), k_hw=(3, 2), lib=lib)
+    t = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=torch.from_numpy(bias),
+        scale=0.45)
+    _close(res.out, t.numpy(), 1e-12, "query 2x3 / key 3x2 index table")
+
+
+def pin_unequal_grids_factorise(lib):
+    """With K = 0 and query / key grids of their own (3x4 queries, 5x2 keys)
+    the scores are rel_h[i, kh] + rel_w[i, kw], so each row of weights, viewed
+    as a Kh x Kw matrix, has rank 1 and equals the outer product of its two
+    marginals (the index itself is pinned by the hand-enumerated table and the
+    worked example)."""
+    r = _rng(17)
+    Qh, Qw, Kh, Kw, d = 3, 4, 5, 2, 3
+    q = r.standard_normal((1, 2, Qh * Qw, d))
+    k = np.zeros((1, 2, Kh * Kw, d))
+    v = r.standard_normal((1, 2, Kh * Kw, d))
+    Rh = r.standard_normal((Qh + Kh - 1, d))
+    Rw = r.standard_normal((Qw + Kw - 1, d))
+    res = oracle.sdpa(q, k, v, 0.3, rel_pos_h=Rh, rel_pos_w=Rw, q_hw=(Qh, Qw), k_hw=(Kh, Kw),
+                      want_weights=True, lib=lib)
+    W = res.weights.reshape(1, 2, Qh * Qw, Kh, Kw)
+    sv = np.linalg.svd(W, compute_uv=False)
+    assert np.all(sv[..., 1] < 1e-12 * sv[..., 0]), "weights not rank-1 over (kh, kw)"
+    _close(np.einsum("...a,...b->...ab", W.sum(-1), W.sum(-2)), W, 1e-12, "outer product of marginals")
 
 
 def pin_factorisation(lib):
@@ -300,6 +351,6 @@ def pin_rows_subset(lib):
 
 ALL_PINS = [pin_hand_cases, pin_weights_sum_to_one, pin_zero_tables_equal_plain,
             pin_row_constant_bias_shift, pin_constant_values, pin_masked_key_inert,
-            pin_index_table_2x3, pin_factorisation, pin_key_permutation, pin_gqa_repeat,
+            pin_index_table_2x3, pin_index_table_q2x3_k3x2, pin_unequal_grids_factorise, pin_factorisation, pin_key_permutation, pin_gqa_repeat,
             pin_window_special_cases, pin_float_and_bool_neutral, pin_torch_library_masks,
             pin_lse_closed_form, pin_rows_subset]

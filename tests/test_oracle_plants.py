@@ -19,6 +19,7 @@ PLANTS = {
     10: "softmax not normalised",
     11: "float mask batch stride ignored",
     12: "boolean mask polarity inverted",
+    13: "rel index shifted by the query grid size instead of the key grid size",
 }
 
 
