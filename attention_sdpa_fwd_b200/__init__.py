@@ -27,7 +27,8 @@ STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
 
 # Every symbol include/sdpa.h declares.
 EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_merge", "sdpa_select_path", "sdpa_fwd_host",
-           "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_strerror", "sdpa_version")
+           "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_selftest_wait_timeout", "sdpa_strerror",
+           "sdpa_version")
 
 
 class SdpaError(RuntimeError):
@@ -66,10 +67,12 @@ def lib():
         L.sdpa_select_path.argtypes = _COMMON + [_i32, _vp, _vp, _vp, _vp, _vp]
         L.sdpa_fwd_split_kv_static.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp]
         L.sdpa_last_device_error.argtypes = [_vp]
+        L.sdpa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, _vp]
         L.sdpa_strerror.argtypes = [_i32]
         L.sdpa_strerror.restype = ctypes.c_char_p
         for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_merge", "sdpa_fwd_host", "sdpa_select_path",
-                     "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_version"):
+                     "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_selftest_wait_timeout",
+                     "sdpa_version"):
             getattr(L, name).restype = _i32
         _lib = L
     return _lib
@@ -129,6 +132,10 @@ def sdpa_fwd_split_kv_static(q, k, v, out, dtype, B, Hq, Hkv, Tq, Tkv, d, scale,
 
 def sdpa_last_device_error(stream) -> int:
     return lib().sdpa_last_device_error(stream)
+
+
+def sdpa_selftest_wait_timeout(limit_ns, stream) -> int:
+    return lib().sdpa_selftest_wait_timeout(limit_ns, stream)
 
 
 def sdpa_strerror(status: int) -> str:

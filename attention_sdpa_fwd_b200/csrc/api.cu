@@ -135,7 +135,6 @@ int build_problem(const void* q, const void* k, const void* v, void* out, sdpa_d
     if (q_hw[0] < 1 || q_hw[1] < 1 || k_hw[0] < 1 || k_hw[1] < 1) return SDPA_ERR_INVALID_ARG;
     if ((long long)q_hw[0] * q_hw[1] != Tq || (long long)k_hw[0] * k_hw[1] != Tkv)
       return SDPA_ERR_INVALID_ARG;
-    if (q_hw[0] != k_hw[0] || q_hw[1] != k_hw[1]) return SDPA_ERR_UNSUPPORTED;
     if (!aligned(rel_pos_h, esz) || !aligned(rel_pos_w, esz)) return SDPA_ERR_MISALIGNED;
     p.use_rel = 1;
     p.rel_h = rel_pos_h; p.rel_w = rel_pos_w;
@@ -394,8 +393,8 @@ extern "C" int sdpa_fwd_host(const void* q, const void* k, const void* v, void* 
   const size_t nk = (size_t)B * Hkv * Tkv * d * esz;
   size_t nrh = 0, nrw = 0, nmask = 0;
   if (pr.p.use_rel) {
-    nrh = (size_t)(2 * pr.p.kh_n - 1) * d * esz;
-    nrw = (size_t)(2 * pr.p.kw_n - 1) * d * esz;
+    nrh = (size_t)(pr.p.qh_n + pr.p.kh_n - 1) * d * esz;
+    nrw = (size_t)(pr.p.qw_n + pr.p.kw_n - 1) * d * esz;
   }
   const bool tensor_mask = mask_kind == SDPA_MASK_ADD_FLOAT || mask_kind == SDPA_MASK_BOOL;
   if (tensor_mask && Tkv > 0) {
@@ -520,6 +519,14 @@ extern "C" int sdpa_fwd_split_kv_static(const void* q, const void* k, const void
   p.err = error_word_ptr();
   if (p.err == nullptr) return SDPA_ERR_CUDA;
   return split_kv_static(p, pr.dtype, stream);
+}
+
+extern "C" int sdpa_selftest_wait_timeout(unsigned long long limit_ns, cudaStream_t stream) {
+  // the wait must end well inside any watchdog: at most the kernels' own 2 s
+  if (limit_ns == 0 || limit_ns > 2000000000ull) return SDPA_ERR_INVALID_ARG;
+  int* err = error_word_ptr();
+  if (err == nullptr) return SDPA_ERR_CUDA;
+  return selftest_wait_timeout(limit_ns, err, stream);
 }
 
 extern "C" int sdpa_last_device_error(cudaStream_t stream) {

@@ -99,6 +99,8 @@ void split_kv_workspace_bytes(const Params& p, size_t* cnt_bytes, size_t* data_b
 cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream_t stream);
 // split-KV on the fixed-size static scratch (no allocation); an sdpa_status
 int split_kv_static(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
+// One bounded mbarrier wait that runs out (nothing arrives); sets *err.
+int selftest_wait_timeout(unsigned long long limit_ns, int* err, cudaStream_t stream);
 int num_sms();
 cudaError_t launch_tc(const Params& p, cudaStream_t stream);
 // persistent form of the tensor-core kernel (one CTA per SM over many short problems)

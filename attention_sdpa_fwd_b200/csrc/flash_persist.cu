@@ -593,6 +593,8 @@ int tc_persist_check(const Params& p, sdpa_dtype_t dtype) {
   if (p.use_rel) {
     if (!(p.kw_n == 14 || p.kw_n == 16)) return SDPA_ERR_UNSUPPORTED;
     if (p.kh_n > kRelH) return SDPA_ERR_UNSUPPORTED;
+    // each table (Qh + Kh - 1, Qw + Kw - 1 rows) within its 32 projection columns
+    if (p.qh_n + p.kh_n - 1 > kRelCols || p.qw_n + p.kw_n - 1 > kRelCols) return SDPA_ERR_UNSUPPORTED;
   }
   if (!al16p(p.out)) return SDPA_ERR_MISALIGNED;
   return SDPA_OK;
@@ -621,8 +623,8 @@ cudaError_t launch_tc_persist(const Params& p, cudaStream_t stream) {
   ok = ok && make_tmap_4d(&a.tk, p.k, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.skt, 2 * p.skh, 2 * p.skb, 64, BN, true);
   ok = ok && make_tmap_4d(&a.tv, p.v, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.svt, 2 * p.svh, 2 * p.svb, 64, BN, true);
   if (p.use_rel) {
-    // 32-row boxes (2*16-1 table rows at most); rows past a table read as zero
-    const uint64_t nh = 2 * p.kh_n - 1, nw = 2 * p.kw_n - 1;
+    // 32-row boxes (Qh + Kh - 1 <= 32 table rows); rows past a table read as zero
+    const uint64_t nh = p.qh_n + p.kh_n - 1, nw = p.qw_n + p.kw_n - 1;
     ok = ok && make_tmap_3d(&a.trh, p.rel_h, bf, 2, p.d, nh, 1, rowb, rowb * nh, 64, kRelCols, true);
     ok = ok && make_tmap_3d(&a.trw, p.rel_w, bf, 2, p.d, nw, 1, rowb, rowb * nw, 64, kRelCols, true);
   }

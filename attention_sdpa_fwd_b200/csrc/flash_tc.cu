@@ -60,13 +60,6 @@ constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-po
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Pairs of score columns whose index satisfies (i & kEmuMask) == kEmuMask take
-// 2^y on the FMA pipe (negative: every exponential on the MUFU unit).
-#ifndef SDPA_EMU_MASK
-#define SDPA_EMU_MASK -1
-#endif
-constexpr int kEmuMask = SDPA_EMU_MASK;
-
 enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3 };
 
 struct TcArgs {
@@ -115,31 +108,6 @@ struct Layout {
   static_assert(kAlloc <= 232448, "shared memory budget");
   static_assert(KW == 0 || (BN % (KW > 0 ? KW : 1) == 0), "key tile must hold whole key-grid rows");
 };
-
-// 2^y for a pair, on the FMA pipe: Cody-Waite reduction y = n + f with
-// n = round(y) (the magic-number add leaves n in the low mantissa bits of t),
-// f in [-1/2, 1/2]; 2^f by the degree-3 minimax polynomial of
-// fit_exp2_poly.py (max relative error 7.5e-5, well under bf16's 2^-9); 2^n
-// added straight into the exponent field.  y is clamped at -125 so the result
-// stays a normal number (callers only use it where no score is -inf).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t y2) {
-  float y0, y1;
-  f2_split(y2, y0, y1);
-  y2 = f2(fmaxf(y0, -125.f), fmaxf(y1, -125.f));
-  const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t t2 = f2_add(y2, f2(kMagic, kMagic));
-  const uint64_t n2 = f2_add(t2, f2(-kMagic, -kMagic));
-  const uint64_t fr = f2_fma(n2, f2(-1.f, -1.f), y2);
-  uint64_t p2 = f2_fma(fr, f2(5.517166906e-02f, 5.517166906e-02f), f2(2.426111222e-01f, 2.426111222e-01f));
-  p2 = f2_fma(p2, fr, f2(6.932609855e-01f, 6.932609855e-01f));
-  p2 = f2_fma(p2, fr, f2(9.999280735e-01f, 9.999280735e-01f));
-  float p0, p1, t0, t1;
-  f2_split(p2, p0, p1);
-  f2_split(t2, t0, t1);
-  const uint32_t r0 = __float_as_uint(t0) * 8388608u + __float_as_uint(p0);  // += n << 23
-  const uint32_t r1 = __float_as_uint(t1) * 8388608u + __float_as_uint(p1);
-  return f2u(r0, r1);
-}
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -737,10 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       }
       // p = 2^(x + goff - m), packed to bf16 pairs in registers first, so that
       // the wait for the previous P.V below comes after the exponentials.
-      // Some pairs take 2^y on the FMA pipe instead of the MUFU unit (only on
-      // tiles that hold no -inf: the polynomial path cannot return an exact 0).
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const bool emu = kEmuMask >= 0 && (MASK == TC_NONE) && (j0 + BN <= args.Tkv);
       uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
       uint32_t pk[BN / 2];
 #pragma unroll
@@ -748,15 +713,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         const int c = 2 * i;
         const float nmo = goff[c / GW] - m_use;
         const uint64_t y2 = f2_add(x2[i], f2(nmo, nmo));
-        float p0, p1;
-        if (kEmuMask >= 0 && emu && (i & kEmuMask) == kEmuMask) {
-          f2_split(exp2_poly2(y2), p0, p1);
-        } else {
-          float lo, hi;
-          f2_split(y2, lo, hi);
-          p0 = ex2_approx(lo);
-          p1 = ex2_approx(hi);
-        }
+        float lo, hi;
+        f2_split(y2, lo, hi);
+        const float p0 = ex2_approx(lo);
+        const float p1 = ex2_approx(hi);
         sum2[i & 1] = f2_add(sum2[i & 1], f2(p0, p1));
         pk[i] = pack_bf16x2(p0, p1);
       }
@@ -995,14 +955,6 @@ cudaError_t dispatch_mask(int mk, const TcArgs& a, dim3 grid, cudaStream_t strea
   return cudaErrorInvalidValue;
 }
 
-template <int D, int BN, int KW, int NS>
-cudaError_t dispatch_mask_rel(int mk, const TcArgs& a, dim3 grid, cudaStream_t stream) {
-  switch (mk) {
-    case TC_NONE: return launch_one<D, BN, KW, TC_NONE, NS>(a, grid, stream);
-    case TC_RANGE: return launch_one<D, BN, KW, TC_RANGE, NS>(a, grid, stream);
-  }
-  return cudaErrorInvalidValue;
-}
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -1018,6 +970,13 @@ int tc_mask_code(const Params& p) {
 }
 
 }  // namespace
+
+// Rows of the larger rel table (Qh + Kh - 1 or Qw + Kw - 1), padded to a
+// multiple of 16: the N of the projection MMAs and the TMA box height.
+static int rel_rows_padded(const Params& p) {
+  const int nh = p.qh_n + p.kh_n - 1, nw = p.qw_n + p.kw_n - 1;
+  return ((nh > nw ? nh : nw) + 15) / 16 * 16;
+}
 
 // Whether the tensor-core kernel takes this (already validated) problem;
 // SDPA_OK, SDPA_ERR_UNSUPPORTED or SDPA_ERR_MISALIGNED.
@@ -1040,9 +999,7 @@ int tc_check(const Params& p, sdpa_dtype_t dtype) {
     if (!(kw == 14 || kw == 16 || kw == 32 || kw == 64)) return SDPA_ERR_UNSUPPORTED;
     if (p.kh_n > kRelHMax) return SDPA_ERR_UNSUPPORTED;
     // the padded tables borrow one K/V stage buffer: at most BN rows
-    const int kmax = p.kh_n > kw ? p.kh_n : kw;
-    if (((2 * kmax - 1) + 15) / 16 * 16 > (kw == 14 ? 112 : 128)) return SDPA_ERR_UNSUPPORTED;
-    if (p.mask_kind == SDPA_MASK_ADD_FLOAT || p.mask_kind == SDPA_MASK_BOOL) return SDPA_ERR_UNSUPPORTED;
+    if (rel_rows_padded(p) > (kw == 14 ? 112 : 128)) return SDPA_ERR_UNSUPPORTED;
     if (!al16(p.rel_h) || !al16(p.rel_w)) return SDPA_ERR_MISALIGNED;
   }
   return SDPA_OK;
@@ -1089,15 +1046,6 @@ void tc_schedule(long long units, int nt, int nsm, bool ranged, bool rel, int* n
       }
     }
   }
-#ifdef SDPA_TUNING
-  if (const char* e = getenv("SDPA_TC_SCHEDULE")) {  // "n_full,n_split" (tuning builds only)
-    int f = 0, sp = 1;
-    if (sscanf(e, "%d,%d", &f, &sp) == 2 && f >= 0 && f <= units && sp >= 1 && sp <= nt && sp <= kMaxSplit) {
-      *n_full = f;
-      *n_split = (f == units) ? 1 : sp;
-    }
-  }
-#endif
 }
 
 cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
@@ -1111,9 +1059,8 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   ok = ok && make_tmap_4d(&a.tk, p.k, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.skt, 2 * p.skh, 2 * p.skb, 64, BN, true);
   ok = ok && make_tmap_4d(&a.tv, p.v, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.svt, 2 * p.svh, 2 * p.svb, 64, BN, true);
   if (p.use_rel) {
-    const int kmax = p.kh_n > p.kw_n ? p.kh_n : p.kw_n;
-    a.rel_n = ((2 * kmax - 1) + 15) / 16 * 16;
-    const uint64_t nh = 2 * p.kh_n - 1, nw = 2 * p.kw_n - 1;
+    a.rel_n = rel_rows_padded(p);
+    const uint64_t nh = p.qh_n + p.kh_n - 1, nw = p.qw_n + p.kw_n - 1;
     ok = ok && make_tmap_3d(&a.trh, p.rel_h, bf, 2, p.d, nh, 1, rowb, rowb * nh, 64, a.rel_n, true);
     ok = ok && make_tmap_3d(&a.trw, p.rel_w, bf, 2, p.d, nw, 1, rowb, rowb * nw, 64, a.rel_n, true);
   }
@@ -1159,10 +1106,10 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
     return dispatch_mask<128, 128, 0, 2>(mk, a, grid, stream);
   }
   switch (p.kw_n) {
-    case 14: return dispatch_mask_rel<64, 112, 14, 3>(mk, a, grid, stream);
-    case 16: return dispatch_mask_rel<64, 128, 16, 2>(mk, a, grid, stream);
-    case 32: return dispatch_mask_rel<64, 128, 32, 2>(mk, a, grid, stream);
-    case 64: return dispatch_mask_rel<64, 128, 64, 2>(mk, a, grid, stream);
+    case 14: return dispatch_mask<64, 112, 14, 3>(mk, a, grid, stream);
+    case 16: return dispatch_mask<64, 128, 16, 2>(mk, a, grid, stream);
+    case 32: return dispatch_mask<64, 128, 32, 2>(mk, a, grid, stream);
+    case 64: return dispatch_mask<64, 128, 64, 2>(mk, a, grid, stream);
   }
   return cudaErrorInvalidValue;
 }

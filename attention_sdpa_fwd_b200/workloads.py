@@ -58,6 +58,11 @@ class Spec:
     def rel(self) -> bool:
         return self.q_hw is not None
 
+    def table_rows(self) -> Tuple[int, int]:
+        """Rows of the rel-pos tables: Qh + Kh - 1 and Qw + Kw - 1 (2*K - 1 for
+        equal query and key grids)."""
+        return self.q_hw[0] + self.k_hw[0] - 1, self.q_hw[1] + self.k_hw[1] - 1
+
     # -- algorithmic work (counts the pages' math, not tile padding) ---------
     def allowed_pairs_per_head(self) -> int:
         """Visible (query, key) pairs of one (b, h) under a causal/sliding mask;
@@ -87,7 +92,7 @@ class Spec:
         e = 4 if self.dtype == torch.float32 else 2
         n = (2 * self.B * self.Hq * self.Tq + 2 * self.B * self.Hkv * self.Tkv) * self.d * e
         if self.rel:
-            n += ((2 * self.k_hw[0] - 1) + (2 * self.k_hw[1] - 1)) * self.d * e
+            n += sum(self.table_rows()) * self.d * e
         if self.mask_kind == MASK_FLOAT:
             n += self.B * self.mask_heads * self.Tq * self.Tkv * e
         if self.mask_kind == MASK_BOOL:
@@ -121,9 +126,9 @@ def make(spec: Spec, seed: Optional[int] = None) -> Workload:
     v = _randn(g, (spec.B, spec.Hkv, spec.Tkv, spec.d), spec.qkv_std).to(dt)
     rh = rw = None
     if spec.rel:
-        kh, kw = spec.k_hw
-        rh = _randn(g, (2 * kh - 1, spec.d), spec.rel_std).to(dt)
-        rw = _randn(g, (2 * kw - 1, spec.d), spec.rel_std).to(dt)
+        nh, nw = spec.table_rows()
+        rh = _randn(g, (nh, spec.d), spec.rel_std).to(dt)
+        rw = _randn(g, (nw, spec.d), spec.rel_std).to(dt)
     mask = None
     if spec.mask_kind == MASK_FLOAT:
         shape = (spec.B, spec.mask_heads, spec.Tq, spec.Tkv)

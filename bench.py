@@ -254,11 +254,17 @@ def auto_path_name(S, spec: W.Spec) -> str:
     return names.get(rc, f"status {rc}")
 
 
-def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, ws: int, path=0):
+def n_input_sets(spec: W.Spec) -> int:
+    """Input sets to rotate so that consecutive launches never find their
+    inputs in the 126 MB L2 (together at least twice its size)."""
+    return min(64, max(2, math.ceil(2 * L2_BYTES / max(spec.bytes(), 1))))
+
+
+def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, ws: int, path=0, sets=None):
     per_set = spec.bytes()
-    nsets = max(2, math.ceil(2 * L2_BYTES / max(per_set, 1)))
-    nsets = min(nsets, 64)
-    sets = make_device_sets(spec, device, nsets, seed_base=spec.seed + 1000 * rank)
+    if sets is None:
+        sets = make_device_sets(spec, device, n_input_sets(spec), seed_base=spec.seed + 1000 * rank)
+    nsets = len(sets)
     stream = torch.cuda.current_stream(device)
     for i in range(warmup):
         launch(S, spec, sets[i % nsets], stream, path)
@@ -287,13 +293,13 @@ def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, w
                 set_bytes=per_set)
 
 
-def time_graph(S, spec: W.Spec, device, launches: int = 40, reps: int = 5):
+def time_graph(S, spec: W.Spec, device, launches: int = 40, reps: int = 5, sets=None):
     """Per-launch device time from CUDA-graph replays of `launches` back-to-back
     launches (rotating input sets): strips the host launch overhead that
     dominates per-launch events for the microsecond-sized workloads."""
-    per_set = spec.bytes()
-    nsets = min(16, max(2, math.ceil(2 * L2_BYTES / max(per_set, 1))))
-    sets = make_device_sets(spec, device, nsets, seed_base=spec.seed)
+    if sets is None:
+        sets = make_device_sets(spec, device, n_input_sets(spec), seed_base=spec.seed)
+    nsets = len(sets)
     side = torch.cuda.Stream(device)
     with torch.cuda.stream(side):
         for i in range(3):
@@ -359,6 +365,62 @@ def time_e2e(S, spec: W.Spec, device, steps: int, warmup: int):
     h2d = sum(x.numel() * x.element_size() for x in (q, k, v, rh, rw, mask_h) if x is not None)
     d2h = out.numel() * out.element_size()
     return ms, h2d, d2h
+
+
+# What bounds each workload's kernel (SURVEY-style work counts live in
+# workloads.Spec.flops / bytes): the dense contractions run against the bf16
+# tensor peak, the streaming shapes against HBM bandwidth, and the two tiny
+# problems (33 KB) are latency-bound and reported in microseconds only.
+BOUND = {"tiny_relpos_f32": "latency", "sam_global": "tensor", "sam_windowed": "hbm",
+         "decoder_token_to_image": "hbm", "decoder_image_to_token": "hbm", "decoder_self": "latency",
+         "gqa_causal": "tensor", "gqa_sliding": "tensor", "gqa_float_mask": "tensor"}
+
+
+def bias_name(spec: W.Spec) -> str:
+    parts = []
+    if spec.rel:
+        parts.append("decomposed rel-pos")
+    if spec.mask_kind != W.MASK_NONE:
+        m = W.MASK_NAMES[spec.mask_kind]
+        if spec.mask_kind == W.MASK_SLIDING:
+            m += f" w={spec.window}"
+        parts.append(m + " mask")
+    return " + ".join(parts) if parts else "none"
+
+
+def dtype_name(spec: W.Spec) -> str:
+    return "bf16" if spec.dtype == torch.bfloat16 else "f32"
+
+
+def per_config_table(S, device, peaks, steps: int):
+    """Every benchmark workload through AUTO: median per-launch CUDA-event time
+    (rotating inputs larger than L2), per-launch time from CUDA-graph replays,
+    and the fraction of the workload's roofline (bf16 burst tensor peak or HBM
+    copy bandwidth) from the graph time."""
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    bf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    table = {}
+    for name, sp in W.SPECS.items():
+        sets = make_device_sets(sp, device, n_input_sets(sp), seed_base=sp.seed + 500)
+        rr = time_workload(S, sp, device, steps, 3, 0, 1, sets=sets)
+        lm = sorted(rr["launch_ms"])[len(rr["launch_ms"]) // 2]
+        gm = time_graph(S, sp, device, launches=20 if sp.flops() > 1e11 else 40, reps=3, sets=sets)
+        del sets
+        torch.cuda.empty_cache()
+        tf = sp.flops() / (gm * 1e-3) / 1e12
+        gbs = sp.bytes() / (gm * 1e-3) / 1e9
+        bound = BOUND.get(name, "tensor")
+        e = dict(path=auto_path_name(S, sp), bias=bias_name(sp), dtype=dtype_name(sp),
+                 us_events_median=lm * 1e3, us_graph=gm * 1e3, flops=sp.flops(), bytes=sp.bytes(),
+                 tflops=tf, gbs=gbs, bound=bound)
+        if bound == "tensor":
+            e.update(frac=tf / bf, peak=bf, peak_unit="TFLOP/s")
+        elif bound == "hbm":
+            e.update(frac=gbs / hbm, peak=hbm, peak_unit="GB/s")
+        else:
+            e.update(frac=None, peak=None, peak_unit=None)
+        table[name] = e
+    return table
 
 
 _WL_CACHE = {}
@@ -461,28 +523,23 @@ def run_ours(args):
     e2e = aggregate_throughput(flops, e2e_ms, ws)
 
     per_config = {}
-    if args.per_config and rank == 0:
-        for name, sp in W.SPECS.items():
-            if name == spec.name:
-                continue
-            rr = time_workload(S, sp, device, max(3, args.steps // 4), 3, 0, 1)
-            lm = sum(rr["launch_ms"]) / len(rr["launch_ms"])
-            gm = time_graph(S, sp, device)
-            hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-            bf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-            per_config[name] = dict(path=auto_path_name(S, sp), ms=lm, graph_ms=gm,
-                                    tflops=sp.flops() / (gm * 1e-3) / 1e12,
-                                    gbs=sp.bytes() / (gm * 1e-3) / 1e9,
-                                    frac_bf16=sp.flops() / (gm * 1e-3) / 1e12 / bf,
-                                    frac_hbm=sp.bytes() / (gm * 1e-3) / 1e9 / hbm)
+    if not args.no_per_config and ws == 1:
+        per_config = per_config_table(S, device, peaks, max(10, args.steps))
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(spec, budget_s=args.cpu_budget)
         cpu.pop("seconds", None)
 
-    achieved = flops / (launch_avg * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    bound = BOUND.get(spec.name, "tensor")
+    if bound == "hbm":
+        achieved = spec.bytes() / (launch_avg * 1e-3) / 1e9
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        r_unit, peak_key = "GB/s", "hbm_gbs (copy)"
+    else:
+        achieved = flops / (launch_avg * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        r_unit, peak_key = "TFLOP/s", "bf16_tflops (burst)"
     khash = kernel_source_hash()
     line = {
         "metric": METRIC,
@@ -495,17 +552,19 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)/sqrt2 q,k,v; rel-pos tables N(0,0.02^2))",
-        "config": {"workload": spec.name, "B": spec.B, "H": spec.Hq, "T": spec.Tq, "head_dim": spec.d,
-                   "grid": list(spec.q_hw) if spec.q_hw else None, "bias": "decomposed rel-pos",
+        "dtype": dtype_name(spec),
+        "data": f"synthetic (seeded normal q, k, v with std {spec.qkv_std:.3g}"
+                + (f"; rel-pos tables std {spec.rel_std}" if spec.rel else "") + ")",
+        "config": {"workload": spec.name, "B": spec.B, "H": spec.Hq, "Hkv": spec.Hkv, "Tq": spec.Tq,
+                   "Tkv": spec.Tkv, "head_dim": spec.d,
+                   "grid": list(spec.q_hw) if spec.q_hw else None, "bias": bias_name(spec),
                    "l2": f"{r['nsets']} rotating input sets of {r['set_bytes'] / 1e6:.1f} MB (> L2)",
                    "parallelism": f"replica x{ws} (independent problems per GPU)"},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_source": f"{peaks_src} bf16_tflops (burst)",
+        "roofline": {"bound": "tensor" if bound != "hbm" else "hbm", "achieved": achieved, "peak": peak,
+                     "unit": r_unit, "frac": achieved / peak, "peak_source": f"{peaks_src} {peak_key}",
                      "traffic": ncu_traffic(khash, spec.name),
                      "flops_per_launch": flops, "launch_ms": launch_avg,
-                     "frac_of_spec_2250": achieved / 2250.0},
+                     "frac_of_spec_sheet": achieved / (7700.0 if bound == "hbm" else 2250.0)},
         "e2e": {"value": e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "cpu_baseline": cpu,
@@ -557,7 +616,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sam_global", choices=sorted(W.SPECS))
-    ap.add_argument("--per-config", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload table (every benchmark workload timed through AUTO)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--profile-launches", type=int, default=0,

@@ -19,7 +19,7 @@
  *     Embeddings": term_h / term_w injected into the scores):
  *         bias[i,j] = q_i . Rh[qh(i) - kh(j) + Kh - 1] + q_i . Rw[qw(i) - kw(j) + Kw - 1]
  *         qh(i) = i / q_hw[1], qw(i) = i % q_hw[1], kh(j) = j / k_hw[1], kw(j) = j % k_hw[1],
- *         Kh = k_hw[0], Kw = k_hw[1];
+ *         Kh = k_hw[0], Kw = k_hw[1] (query and key grids may differ, see sdpa_fwd);
  *   - mask is one of the Axon :mask forms (Axon PR, :mask option) -- causal
  *     with an offset, a sliding window with an offset, or a runtime additive
  *     float / boolean tensor broadcast to [B, Hq, Tq, Tkv] (mlx issue: the
@@ -83,8 +83,8 @@ typedef enum {
   SDPA_OK = 0,
   SDPA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, Hq % Hkv != 0, aliasing, ... */
   SDPA_ERR_UNSUPPORTED = -2,  /* legal request this build does not implement (d not in
-                                 {16,64,128}, rel-pos with q_hw != k_hw, path forced
-                                 onto a kernel that cannot take the problem) */
+                                 {16,64,128}, path forced onto a kernel that cannot
+                                 take the problem) */
   SDPA_ERR_MISALIGNED = -3,   /* a pointer or stride breaks the 16-byte rule of the
                                  forced tensor-core path */
   SDPA_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (launch, copy) */
@@ -121,13 +121,17 @@ typedef enum {
  *   scale        : score scale, finite (the Axon default 1/sqrt(d) is applied
  *                  by the Python binding, not here).
  *   mask_kind, mask_ptr : sdpa_mask_kind_t and a host sdpa_mask_t* (see above).
- *   rel_pos_h, rel_pos_w : device tables [2*k_hw[0]-1, d] and [2*k_hw[1]-1, d]
- *                  in the I/O dtype, shared by every batch and head; both NULL
- *                  disables the bias, exactly one NULL is INVALID_ARG.
+ *   rel_pos_h, rel_pos_w : device tables [q_hw[0]+k_hw[0]-1, d] and
+ *                  [q_hw[1]+k_hw[1]-1, d] (2*K-1 rows each when the grids are
+ *                  equal) in the I/O dtype, shared by every batch and head;
+ *                  both NULL disables the bias, exactly one NULL is INVALID_ARG.
  *   q_hw, k_hw   : host int[2] patch grids (height, width) with
  *                  q_hw[0]*q_hw[1] == Tq and k_hw[0]*k_hw[1] == Tkv; required
- *                  with rel-pos, ignored otherwise.  q_hw != k_hw is
- *                  UNSUPPORTED (the pages give the equal-size formula only).
+ *                  with rel-pos, ignored otherwise.  The grids may differ:
+ *                  the bias formula above is read with qh, qw from the query
+ *                  grid and kh, kw and the shifts Kh-1, Kw-1 from the key
+ *                  grid, so table row qh-kh+Kh-1 covers offsets -(Kh-1) ..
+ *                  Qh-1 (no interpolation of resized tables).
  *   stream       : CUDA stream the work is enqueued on.
  */
 int sdpa_fwd(const void* q, const void* k, const void* v, void* out, sdpa_dtype_t dtype,
@@ -276,6 +280,17 @@ int sdpa_fwd_split_kv_static(const void* q, const void* k, const void* v, void* 
    wait since the last call (its output is then undefined), or SDPA_ERR_CUDA
    when the synchronisation itself failed. */
 int sdpa_last_device_error(cudaStream_t stream);
+
+/* Self-test of the failure detection above (the pages have no counterpart;
+   it checks this library's own error path).  Enqueues on `stream` one kernel
+   whose single thread waits, bounded by limit_ns nanoseconds of %globaltimer,
+   on an mbarrier that nothing arrives on -- the same bounded wait every
+   tensor-core kernel uses -- and so sets the device error word exactly as an
+   expired wait inside a forward call would.  The next sdpa_last_device_error
+   then returns SDPA_ERR_TIMEOUT and clears the word.  No fault, trap or hang
+   is involved and the CUDA context stays usable.  limit_ns must be in
+   (0, 2e9]: SDPA_ERR_INVALID_ARG otherwise, before any launch. */
+int sdpa_selftest_wait_timeout(unsigned long long limit_ns, cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* sdpa_strerror(int status);

@@ -106,12 +106,24 @@ def test_auto_takes_persistent_form_for_many_short_problems(L):
     (dict(rh=0x600000), -1),                 # only one table
     (dict(rh=0x600000, rw=0x700000), -1),    # tables without grids
     (dict(rh=0x600000, rw=0x700000, q_hw=(2, 3), k_hw=(2, 4)), -1),   # grid != Tq
-    (dict(rh=0x600000, rw=0x700000, q_hw=(2, 4), k_hw=(4, 2)), -2),   # q_hw != k_hw
     (dict(rh=0x600000, rw=0x700000, q_hw=(0, 8), k_hw=(0, 8)), -1),
     (dict(rh=0x600001, rw=0x700000, q_hw=(2, 4), k_hw=(2, 4)), -3),
 ])
 def test_invalid_arguments_rejected(L, kw, code):
     assert sel(**kw) == code
+
+
+def test_unequal_query_and_key_grids_are_valid(L):
+    """Rel-pos with query and key grids of their own (tables of Qh+Kh-1 and
+    Qw+Kw-1 rows) is a valid problem; the tensor-core path takes it when the
+    key-grid width is one it specialises and both tables fit its 128 rows."""
+    rh, rw = 0x600000, 0x700000
+    far = dict(q=0x10000000, k=0x20000000, v=0x30000000, out=0x40000000)
+    assert sel(**far, rh=rh, rw=rw, Tq=8, Tkv=8, q_hw=(2, 4), k_hw=(4, 2)) == S.PATH_EXACT
+    assert sel(**far, rh=rh, rw=rw, Tq=64, Tkv=256, q_hw=(8, 8), k_hw=(16, 16)) == S.PATH_TCGEN05
+    assert sel(**far, rh=rh, rw=rw, Tq=4096, Tkv=1024, q_hw=(64, 64), k_hw=(32, 32)) == S.PATH_TCGEN05
+    # 100 + 64 - 1 table rows do not fit the 128-row projection
+    assert sel(**far, rh=rh, rw=rw, Tq=6400, Tkv=4096, q_hw=(100, 64), k_hw=(64, 64)) == S.PATH_EXACT
 
 
 def test_empty_problems_are_valid(L):

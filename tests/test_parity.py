@@ -102,6 +102,32 @@ CASES = [
     # first unit (the hand-over that waits for the unit two back)
     S_("persist_relpos_14x14_deep", BF16, 80, 6, 6, 196, 196, 64, q_hw=(14, 14), k_hw=(14, 14), rel_std=0.5,
        seed=55),
+    # rel-pos combined with an additive float or a boolean mask tensor
+    S_("relpos_float_bf16_d64_12x16", BF16, 2, 2, 1, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5,
+       mask_kind=W.MASK_FLOAT, mask_std=1.0, mask_neg_inf_frac=0.2, mask_heads=2, seed=70),
+    S_("relpos_bool_bf16_d64_20x14", BF16, 1, 3, 3, 280, 280, 64, q_hw=(20, 14), k_hw=(20, 14), rel_std=0.5,
+       mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.4, mask_heads=1, seed=71),
+    S_("relpos_float_bf16_d64_5x64", BF16, 1, 2, 2, 320, 320, 64, q_hw=(5, 64), k_hw=(5, 64), rel_std=0.5,
+       mask_kind=W.MASK_FLOAT, mask_std=2.0, mask_neg_inf_frac=0.1, mask_heads=1, seed=72),
+    S_("relpos_bool_bf16_d64_8x32_strong", BF16, 1, 2, 2, 256, 256, 64, q_hw=(8, 32), k_hw=(8, 32), rel_std=1.0,
+       mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.5, mask_heads=2, seed=73),
+    S_("relpos_float_f32_d16_6x6", F32, 1, 2, 2, 36, 36, 16, q_hw=(6, 6), k_hw=(6, 6), rel_std=0.5,
+       mask_kind=W.MASK_FLOAT, mask_std=1.0, mask_neg_inf_frac=0.2, mask_heads=2, seed=74),
+    # rel-pos with query and key grids of their own (tables of Qh+Kh-1 and Qw+Kw-1 rows)
+    S_("relpos_qk_bf16_d64_q8x16_k12x16", BF16, 2, 2, 2, 128, 192, 64, q_hw=(8, 16), k_hw=(12, 16), rel_std=0.5,
+       seed=80),
+    S_("relpos_qk_bf16_d64_q10x14_k14x14", BF16, 3, 2, 2, 140, 196, 64, q_hw=(10, 14), k_hw=(14, 14),
+       rel_std=0.5, seed=81),
+    S_("relpos_qk_bf16_d64_q16x32_k8x32", BF16, 1, 3, 3, 512, 256, 64, q_hw=(16, 32), k_hw=(8, 32), rel_std=0.5,
+       seed=82),
+    S_("relpos_qk_bf16_d64_q64x64_k16x16", BF16, 1, 2, 2, 4096, 256, 64, q_hw=(64, 64), k_hw=(16, 16),
+       rel_std=0.3, seed=83),
+    S_("relpos_qk_bf16_d64_q3x64_k5x64_causal", BF16, 1, 2, 2, 192, 320, 64, q_hw=(3, 64), k_hw=(5, 64),
+       rel_std=0.5, mask_kind=W.MASK_CAUSAL, offset=100, seed=84),
+    S_("relpos_qk_bf16_d16_q5x7_k3x9", BF16, 2, 2, 1, 35, 27, 16, q_hw=(5, 7), k_hw=(3, 9), rel_std=0.5, seed=85),
+    S_("relpos_qk_f32_d64_q4x6_k6x4", F32, 1, 2, 2, 24, 24, 64, q_hw=(4, 6), k_hw=(6, 4), rel_std=0.5, seed=86),
+    S_("relpos_qk_bf16_d64_q14x14_k7x14_strong", BF16, 40, 2, 2, 196, 98, 64, q_hw=(14, 14), k_hw=(7, 14),
+       rel_std=1.0, seed=87),
 ]
 CASE_IDS = [c.name for c in CASES]
 
@@ -121,15 +147,14 @@ def applicable(path: str, sp: W.Spec) -> bool:
             kh, kw = sp.k_hw
             bn = 112 if kw == 14 else 128
             return (sp.d == 64 and kw in (14, 16, 32, 64) and kh <= 64
-                    and ((2 * max(kh, kw) - 1) + 15) // 16 * 16 <= bn
-                    and sp.mask_kind in (W.MASK_NONE, W.MASK_CAUSAL, W.MASK_SLIDING))
+                    and (max(sp.table_rows()) + 15) // 16 * 16 <= bn)
         return True
     if path in ("small_d", "split_kv"):
         return sp.d == 16 and not sp.rel
     if path == "tc_persistent":
         if sp.d != 64 or sp.mask_kind != W.MASK_NONE:
             return False
-        return (not sp.rel) or (sp.k_hw[1] in (14, 16) and sp.k_hw[0] <= 16)
+        return (not sp.rel) or (sp.k_hw[1] in (14, 16) and sp.k_hw[0] <= 16 and max(sp.table_rows()) <= 32)
     return False
 
 
