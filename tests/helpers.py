@@ -41,8 +41,8 @@ def assert_gates(got, ref, dtype, what="", strong=False):
     """The stated gates.  ``strong`` (bias-dominated companions only, never the
     stated workloads) replaces the flat bf16 max gate by 2e-2 + 2^-7*|ref| per
     element: there the output sits on single value rows of magnitude up to ~5,
-    where bf16 output rounding alone is up to 2^-9*|ref| and the bf16 rounding
-    of P adds at most 2^-8*|ref|."""
+    where bf16 output rounding (unit roundoff 2^-8) is up to 2^-8*|ref| and the
+    bf16 rounding of P adds at most another 2^-8*|ref|."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
