@@ -60,13 +60,6 @@ constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-po
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-#ifndef SDPA_MMA2
-#define SDPA_MMA2 0
-#endif
-#ifndef SDPA_PINGPONG
-#define SDPA_PINGPONG 0
-#endif
-
 enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3 };
 
 struct TcArgs {
@@ -109,7 +102,7 @@ struct Layout {
   static constexpr int oV = oK + NS * kKVBytes;
   static constexpr int oRel = oV + NS * kKVBytes;
   static constexpr int oBar = oRel + kRelRows * 256 * 4;
-  static constexpr int kBars = 4 * NS + 28;
+  static constexpr int kBars = 4 * NS + 20;
   static constexpr int kTotal = oBar + kBars * 8 + 32;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -134,11 +127,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   // S_t(j+2) goes into that buffer right after O_t += P_t(j).V_j (in issue
   // order), so the next score tile is always computed one tile ahead.
   constexpr bool kSDB = (D == 128 && BN == 64);
-  // With P in columns of its own, each query tile gets an MMA warp of its own
-  // (warp 9 for A, warp 10 for B): S_t(j+1) is issued as soon as softmax t has
-  // read S_t(j), whatever the other tile's softmax is doing.
-  constexpr bool kMma2 = kPSep && SDPA_MMA2;
-  constexpr bool kPing = kMma2 && SDPA_PINGPONG;
   constexpr bool kRwInSmem = KW >= 32;  // large key-grid width: rel_w re-read per tile
   constexpr int kRwSwz = KW >= 64 ? 15 : 7;  // float4-index XOR swizzle of those rows (conflict-free)
   extern __shared__ uint8_t smem_raw[];
@@ -172,10 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   // of its waiter
   uint64_t* s_odd = q_full + 16;         // [2]
   uint64_t* p_odd = q_full + 18;         // [2]   (128 arrivals)
-  // exponential-phase hand-over between the two softmax warps of a
-  // sub-partition (warp w of tile A, warp w + 4 of tile B): A -> B and B -> A
-  uint64_t* pp_ab = q_full + 20;         // [4]
-  uint64_t* pp_ba = q_full + 24;         // [4]
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + L::kBars);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
 
@@ -228,14 +212,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     mbar_init(&s_free[1], kRowsPerTile);
     mbar_init(&p_odd[0], kRowsPerTile);
     mbar_init(&p_odd[1], kRowsPerTile);
-    if (kMma2) {
-      // both MMA warps commit once per use of a K / V stage, and once at the end
-      for (int i = 0; i < NS; ++i) {
-        mbar_init(&k_empty[i], 2);
-        mbar_init(&v_empty[i], 2);
-      }
-      mbar_init(fin, 2);
-    }
     fence_mbar_init();
     if (n_tiles > 0) {
       // Q (and the rel tables) and the first K tile go out before the TMEM
@@ -332,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           mbar_wait(&v_full[jj % NS], (jj / NS) & 1, nullptr, args.err);
       }
     }
-  } else if (warp == 9 || (kMma2 && warp == 10)) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop (every wait is warp-uniform) and one elected
     // lane issues each instruction: measured faster than lane 0 running it
@@ -365,8 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         for (int kk = 0; kk < BN / 16; ++kk)
           mma_ts_x(d_tm, a_tm + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (!first) || kk > 0);
       };
-      const int mt = warp - 9;  // kMma2: the query tile this warp issues for
-      if (ok && KW > 0 && (!kMma2 || mt == 0)) {
+      if (ok && KW > 0) {
         // rel projections: Ph_t -> cols [256t, 256t+rel_n), Pw_t -> [256t+128, 256t+128+rel_n)
         const uint32_t id_rel = idesc_bf16_f32(128, args.rel_n, false, false);
         const uint64_t drh = dk + (uint64_t)(((NS - 1) * L::kKVBytes) >> 4);
@@ -379,45 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
               mma_ss_x(tbase + t * 256 + w * 128, dq + (uint64_t)((t * L::kQBytes + kk * 32) >> 4),
                      (w == 0 ? drh : drw) + (uint64_t)((kk * 32) >> 4), id_rel, kk > 0);
         mma_commit_x(rel_mma);
-      }
-      if (ok && KW > 0) ok = wait_x(mbar_wait(rel_read, 0, abort_v, args.err));
-      if constexpr (kMma2) {
-        // tile mt alone: S(0); then per key tile S(j+1) as soon as softmax has
-        // read S(j), and O += P(j).V_j as soon as it has written P(j)
-        const int t = mt;
-        if (ok) ok = wait_x(mbar_wait(&k_full[0], 0, abort_v, args.err));
-        if (ok) {
-          tc_fence_after();
-          qk(t, 0);
-          mma_commit_x(&s_full[t]);
-          mma_commit_x(&k_empty[0]);
-        }
-        for (int jj = 0; jj < n_tiles && ok; ++jj) {
-          const int s = jj % NS;
-          const int s1 = (jj + 1) % NS;
-          if (jj + 1 < n_tiles) {
-            ok = wait_x(mbar_wait(&k_full[s1], ((jj + 1) / NS) & 1, abort_v, args.err));
-            if (ok) ok = wait_x(mbar_wait(&s_free[t], jj & 1, abort_v, args.err));
-            if (!ok) break;
-            tc_fence_after();
-            qk(t, s1);
-            mma_commit_x(&s_full[t]);
-            mma_commit_x(&k_empty[s1]);
-          }
-          ok = wait_x(mbar_wait(&v_full[s], (jj / NS) & 1, abort_v, args.err));
-          if (ok) ok = wait_x(mbar_wait(&p_full[t], jj & 1, abort_v, args.err));
-          if (!ok) break;
-          tc_fence_after();
-          pv(t, s, jj == 0);
-          mma_commit_x(&o_ready[t]);
-          mma_commit_x(&v_empty[s]);
-        }
-        mma_commit_x(&o_done[t]);
-        if (mt == 1) mma_commit_x(fin);  // warp 9 commits its own at teardown
+        ok = wait_x(mbar_wait(rel_read, 0, abort_v, args.err));
       }
       // prologue: S_A(0), S_B(0)
-      if (!kMma2 && ok) ok = wait_x(mbar_wait(&k_full[0], 0, abort_v, args.err));
-      if (!kMma2 && ok) {
+      if (ok) ok = wait_x(mbar_wait(&k_full[0], 0, abort_v, args.err));
+      if (ok) {
         tc_fence_after();
         qk(0, 0);
         mma_commit_x(&s_full[0]);
@@ -467,8 +408,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
             mma_commit_x(&k_empty[s2]);
           }
         }
-      } else if constexpr (kMma2) {
-        // issued above
       } else if constexpr (kPSep) {
         // A and B alternate: S_A(j+1), O_A += P_A(j).V_j, S_B(j+1), O_B += P_B(j).V_j
         for (int jj = 0; jj < n_tiles && ok; ++jj) {
@@ -536,10 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           }
         }
       }
-      if (!kMma2) {
-        mma_commit_x(&o_done[0]);
-        mma_commit_x(&o_done[1]);
-      }
+      mma_commit_x(&o_done[0]);
+      mma_commit_x(&o_done[1]);
     }
   }
   } else {
@@ -766,17 +703,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         l_run *= alpha;
         m_run = m_new;
       }
-      if constexpr (kPing) {
-        // the two softmax warps of this sub-partition take turns at their
-        // exponentials (A of tile j, B of tile j, A of tile j+1, ...), so that
-        // one works on the MUFU while the other does everything else
-        if (t == 0) {
-          if (jj > 0) ok = __all_sync(0xffffffffu, mbar_wait(&pp_ba[warp & 3], (jj - 1) & 1, abort_v, args.err));
-        } else {
-          ok = __all_sync(0xffffffffu, mbar_wait(&pp_ab[warp & 3], jj & 1, abort_v, args.err));
-        }
-        if (!ok) break;
-      }
       // p = 2^(x + goff - m), packed to bf16 pairs in registers first, so that
       // the wait for the previous P.V below comes after the exponentials.
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
@@ -799,10 +725,6 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
         f2_split(sum2[0], a0, a1);
         f2_split(sum2[1], b0, b1);
         l_run += (a0 + a1) + (b0 + b1);
-      }
-      if constexpr (kPing) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(t == 0 ? &pp_ab[warp & 3] : &pp_ba[warp & 3]);
       }
       if constexpr (kPSep) {
         // O_t += P_t(j-1).V_{j-1} must be complete before O_t is rescaled or P_t is overwritten
