@@ -367,6 +367,35 @@ def time_e2e(S, spec: W.Spec, device, steps: int, warmup: int):
     return ms, h2d, d2h
 
 
+def time_pinned_copies(device, h2d_bytes: int, d2h_bytes: int, reps: int = 10):
+    """The box's own floor for the host-buffer call: plain pinned copies of the
+    same byte counts (one upload of h2d_bytes, one download of d2h_bytes), on
+    one stream, timed with CUDA events (median of reps)."""
+    up_h = torch.empty(h2d_bytes, dtype=torch.uint8).pin_memory()
+    down_h = torch.empty(d2h_bytes, dtype=torch.uint8).pin_memory()
+    up_d = torch.empty(h2d_bytes, dtype=torch.uint8, device=device)
+    down_d = torch.empty(d2h_bytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def med(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(device)
+        ts = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            ts.append(a.elapsed_time(b))
+        return sorted(ts)[len(ts) // 2]
+    up_ms = med(lambda: up_d.copy_(up_h, non_blocking=True))
+    down_ms = med(lambda: down_h.copy_(down_d, non_blocking=True))
+    return up_ms, down_ms
+
+
 # What bounds each workload's kernel (SURVEY-style work counts live in
 # workloads.Spec.flops / bytes): the dense contractions run against the bf16
 # tensor peak, the streaming shapes against HBM bandwidth, and the two tiny
@@ -476,7 +505,7 @@ def run_profile_launches(args):
     import attention_sdpa_fwd_b200 as S
     S.lib()
     spec = W.SPECS[args.workload]
-    spec = W.scaled(spec, B=spec.B * args.batch_mult)
+    spec = W.scaled(spec, B=args.batch if args.batch > 0 else spec.B * args.batch_mult)
     st = make_device_sets(spec, device, 1, seed_base=spec.seed)[0]
     stream = torch.cuda.current_stream(device)
     for _ in range(args.profile_launches):
@@ -521,6 +550,7 @@ def run_ours(args):
     e2e_ms, h2d, d2h = time_e2e(S, spec, device, max(3, min(args.steps, 20)), 2)
     e2e_ms, = max_over_ranks([e2e_ms], device)
     e2e = aggregate_throughput(flops, e2e_ms, ws)
+    up_ms, down_ms = time_pinned_copies(device, int(h2d), int(d2h))
 
     per_config = {}
     if not args.no_per_config and ws == 1:
@@ -566,7 +596,11 @@ def run_ours(args):
                      "flops_per_launch": flops, "launch_ms": launch_avg,
                      "frac_of_spec_sheet": achieved / (7700.0 if bound == "hbm" else 2250.0)},
         "e2e": {"value": e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
+                "ms_per_step": e2e_ms,
+                # plain pinned copies of the same bytes on this machine: the transfer floor of the call
+                "pinned_upload_ms": up_ms, "pinned_download_ms": down_ms,
+                "pinned_h2d_gbs": h2d / (up_ms * 1e-3) / 1e9, "pinned_d2h_gbs": d2h / (down_ms * 1e-3) / 1e9,
+                "ms_over_serial_copy_floor": e2e_ms / (up_ms + down_ms)},
         "cpu_baseline": cpu,
         "gpu_launches": args.steps,
         "clocks": clocks,
@@ -624,6 +658,8 @@ def main():
                     help="only run this many untimed launches (for ncu) and exit")
     ap.add_argument("--batch-mult", type=int, default=1,
                     help="with --profile-launches: multiply the workload's batch")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="with --profile-launches: set the workload's batch (overrides --batch-mult)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
