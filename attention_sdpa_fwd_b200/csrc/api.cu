@@ -355,8 +355,12 @@ extern "C" int sdpa_select_path(const void* q, const void* k, const void* v, voi
 namespace sdpa {
 namespace {
 
-// Slabs the host entry point pipelines a problem into.
-constexpr int kHostChunks = 6;
+// Slabs the host entry point pipelines a problem into: three measured best
+// for SAM global attention (545 us per call against 568 with six and 608
+// with one, on one B200 machine): fewer slabs overlap less of the uploads with
+// the kernels, more slabs pay a fixed cost per copy and run kernels too
+// small to fill the GPU.
+constexpr int kHostChunks = 3;
 
 // Device staging buffer of sdpa_fwd_host, one per device, grown on demand,
 // with the two copy streams and the events that order the pipeline.

@@ -285,7 +285,7 @@ def test_mixed_schedule(sp):
 
 
 HOST_CASES = [
-    # whole-batch slabs (B >= 6), per-head float mask with -inf entries
+    # whole-batch slabs (B at least the slab count), per-head float mask with -inf entries
     S_("host_batches_float_mask", BF16, 7, 4, 2, 200, 150, 64, mask_kind=W.MASK_FLOAT, mask_std=1.0,
        mask_neg_inf_frac=0.2, mask_heads=4, seed=60),
     # head slabs covering whole GQA groups (group of 4)
