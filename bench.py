@@ -421,6 +421,36 @@ def dtype_name(spec: W.Spec) -> str:
     return "bf16" if spec.dtype == torch.bfloat16 else "f32"
 
 
+def time_copy_floor(device, nbytes: float, launches: int = 40, reps: int = 3) -> float:
+    """Per-copy device time (us) of a plain device-to-device copy that reads
+    and writes nbytes / 2 each, in CUDA-graph replays of back-to-back copies
+    over rotating buffers larger than L2 in all: the practical floor of a
+    memory-bound launch of that much traffic on this GPU."""
+    n = max(16, int(nbytes / 2) // 16 * 16)
+    nbuf = min(16, max(2, math.ceil(2 * L2_BYTES / n)))
+    src = [torch.empty(n, dtype=torch.uint8, device=device) for _ in range(nbuf)]
+    dst = [torch.empty(n, dtype=torch.uint8, device=device) for _ in range(nbuf)]
+    side = torch.cuda.Stream(device)
+    with torch.cuda.stream(side):
+        for i in range(3):
+            dst[i % nbuf].copy_(src[i % nbuf])
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(launches):
+            dst[i % nbuf].copy_(src[i % nbuf])
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / (reps * launches) * 1e3
+
+
 def per_config_table(S, device, peaks, steps: int):
     """Every benchmark workload through AUTO: median per-launch CUDA-event time
     (rotating inputs larger than L2), per-launch time from CUDA-graph replays,
@@ -446,6 +476,10 @@ def per_config_table(S, device, peaks, steps: int):
             e.update(frac=tf / bf, peak=bf, peak_unit="TFLOP/s")
         elif bound == "hbm":
             e.update(frac=gbs / hbm, peak=hbm, peak_unit="GB/s")
+            # context for the HBM fraction of a few-MB launch: a plain copy of the same traffic
+            cu = time_copy_floor(device, sp.bytes())
+            e.update(copy_floor_us=cu, copy_floor_frac_hbm=sp.bytes() / (cu * 1e-6) / 1e9 / hbm,
+                     us_graph_over_copy_floor=gm * 1e3 / cu)
         else:
             e.update(frac=None, peak=None, peak_unit=None)
         table[name] = e
