@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "softmax_tile.cuh"
 #include "tmap.h"
 
 namespace sdpa {
@@ -448,19 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
             }
         }
 
-        // row max: three-input max over pairs, four independent chains per group
-        float mx = -INFINITY;
-#pragma unroll
-        for (int gi = 0; gi < NG; ++gi) {
-          float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int i = 0; i < GW / 2; ++i) {
-            float lo, hi;
-            f2_split(x2[gi * GW / 2 + i], lo, hi);
-            a[i & 3] = max3(a[i & 3], lo, hi);
-          }
-          mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) + goff[gi]);
-        }
+        const float mx = tile::row_max<NG, GW>(x2, goff);
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + kRescaleThreshold;  // false while both are -inf
         float alpha = 1.f;
@@ -472,24 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
         // p = 2^(x + goff - m) packed to bf16 pairs in registers, so that the
         // wait for the previous P.V comes after the exponentials
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        uint64_t sum2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
         uint32_t pk[BN / 2];
-#pragma unroll
-        for (int i = 0; i < BN / 2; ++i) {
-          const float nmo = goff[(2 * i) / GW] - m_use;
-          const uint64_t y2 = f2_add(x2[i], f2(nmo, nmo));
-          float lo, hi;
-          f2_split(y2, lo, hi);
-          const float p0 = ex2_approx(lo), p1 = ex2_approx(hi);
-          sum2[i & 1] = f2_add(sum2[i & 1], f2(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        {
-          float a0, a1, b0, b1;
-          f2_split(sum2[0], a0, a1);
-          f2_split(sum2[1], b0, b1);
-          l_run += (a0 + a1) + (b0 + b1);
-        }
+        l_run += tile::exp_pack<BN, GW>(x2, goff, m_use, pk);
         // O_t += P_t(g-1).V must be complete before O_t is rescaled or P_t
         // overwritten (for a unit's first tile the previous epilogue waited)
         if (j > 0) {
@@ -497,20 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
           if (!ok) break;
           tc_fence_after();
         }
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O_t row *= alpha (warp-collective; alpha is 1 where the max did not move)
-#pragma unroll
-          for (int c0 = 0; c0 < kD; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(o_addr + c0, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(o_addr + c0, r);
-          }
-        }
-#pragma unroll
-        for (int c0 = 0; c0 < BN / 2; c0 += 8) tmem_st8p(p_addr + c0, pk + c0);
+        if (j > 0 && __any_sync(0xffffffffu, need)) tile::rescale_o<kD>(o_addr, alpha);  // O_t row *= alpha
+        tile::store_p<BN>(p_addr, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[t]);
@@ -521,26 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
       ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (it * nt + nt - 1) & 1, abort_v, args.err));
       if (!ok) break;
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (long long)u.b * args.sob +
                             (long long)u.h * args.soh + qi * args.sot;
-#pragma unroll
-      for (int c0 = 0; c0 < kD; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(o_addr + c0, r);
-        tmem_wait_ld();
-        if (row_valid) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[c + 0]) * inv, __uint_as_float(r[c + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(r[c + 2]) * inv, __uint_as_float(r[c + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(r[c + 4]) * inv, __uint_as_float(r[c + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(r[c + 6]) * inv, __uint_as_float(r[c + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c0 + c) = v;
-          }
-        }
-      }
+      tile::store_o_row<kD>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, orow, row_valid);
       if (row_valid && args.lse)
         args.lse[((long long)u.b * args.Hq + u.h) * args.Tq + qi] =
             l_run > 0.f ? m_run * kLn2 + logf(l_run) : -INFINITY;

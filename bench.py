@@ -179,7 +179,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # sources of the tensor-core kernel the bench times (the traffic figure in
 # profiles/traffic.json is valid only for these exact sources)
-TC_SOURCES = ("flash_tc.cu", "common.cuh", "sm100.cuh", "tmap.h")
+TC_SOURCES = ("flash_tc.cu", "common.cuh", "sm100.cuh", "softmax_tile.cuh", "tmap.h")
 
 
 def kernel_source_hash() -> str:
