@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
   extern __shared__ float4 cl_smem[];
   float4 (*sk)[D16 / 4] = reinterpret_cast<float4 (*)[D16 / 4]>(cl_smem);
   float4 (*sv)[D16 / 4] = reinterpret_cast<float4 (*)[D16 / 4]>(cl_smem + kClusterChunk * (D16 / 4));
-  float* part_s = reinterpret_cast<float*>(cl_smem + 2 * kClusterChunk * (D16 / 4));  // [Tq][kPartStride]
+  float* part_s = reinterpret_cast<float*>(cl_smem + 2 * kClusterChunk * (D16 / 4));  // [Tq][2 halves][kPartStride]
   cg::cluster_group cluster = cg::this_cluster();
   const int part = (int)cluster.block_rank(), h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.group;
@@ -412,109 +412,125 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl = p.scale * kLog2e;
-  for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, i);
-    float q[D16];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
-    const long long mrow = (long long)b * p.msb + (long long)h * p.msh + (long long)i * p.msq;
-    // this lane's keys (lane, lane + 32, ...), in two halves of eight to
-    // bound the registers: scores, running max, then the sums
-    float m = -INFINITY, l = 0.f, acc[D16];
+  // Warp w takes two query rows, 2 (w & 3) + 8 r and the next, over one half
+  // of the part's keys (w >> 2): every K and V row read from shared memory
+  // serves two query rows, and each row's two key halves become two partials.
+  const int kh = warp >> 2;
+  for (int i0 = 2 * (warp & 3); i0 < p.Tq; i0 += 8) {
+    const int ir[2] = {i0, min(i0 + 1, p.Tq - 1)};
+    const bool live1 = i0 + 1 < p.Tq;
+    float q[2][D16];
+    long long mrow[2];
 #pragma unroll
-    for (int c = 0; c < D16; ++c) acc[c] = 0.f;
+    for (int r = 0; r < 2; ++r) {
+      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, ir[r]);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q[r]);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q[r] + 8);
+      mrow[r] = (long long)b * p.msb + (long long)h * p.msh + (long long)ir[r] * p.msq;
+    }
+    // this lane's eight keys of the half (lane + 32 u): scores of both rows,
+    // their maxima, then the sums
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, acc[2][D16];
 #pragma unroll
-    for (int half = 0; half < kClusterChunk / 256; ++half) {
-      float sc[8];
-      float cm = -INFINITY;
+    for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = lane + 32 * (half * 8 + u);
-        float x = -INFINITY;
-        if (t < n) {
-          x = 0.f;
+      for (int c = 0; c < D16; ++c) acc[r][c] = 0.f;
+    float sc[2][8];
 #pragma unroll
-          for (int c = 0; c < D16; c += 4) {
-            const float4 k4 = sk[t][(c / 4) ^ ((t >> 1) & 3)];
-            x = fmaf(q[c], k4.x, fmaf(q[c + 1], k4.y, fmaf(q[c + 2], k4.z, fmaf(q[c + 3], k4.w, x))));
-          }
-          x = x * sl + mask_term(p, mrow, i, j0 + t);
+    for (int u = 0; u < 8; ++u) {
+      const int t = lane + 32 * (kh * 8 + u);
+      float x0 = -INFINITY, x1 = -INFINITY;
+      if (t < n) {
+        x0 = 0.f;
+        x1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < D16; c += 4) {
+          const float4 k4 = sk[t][(c / 4) ^ ((t >> 1) & 3)];
+          x0 = fmaf(q[0][c], k4.x, fmaf(q[0][c + 1], k4.y, fmaf(q[0][c + 2], k4.z, fmaf(q[0][c + 3], k4.w, x0))));
+          x1 = fmaf(q[1][c], k4.x, fmaf(q[1][c + 1], k4.y, fmaf(q[1][c + 2], k4.z, fmaf(q[1][c + 3], k4.w, x1))));
         }
-        sc[u] = x;
-        cm = fmaxf(cm, x);
+        x0 = x0 * sl + mask_term(p, mrow[0], ir[0], j0 + t);
+        x1 = x1 * sl + mask_term(p, mrow[1], ir[1], j0 + t);
       }
-      if (cm == -INFINITY) continue;
-      if (cm > m) {
-        const float corr = sm100::ex2_approx(m - cm);  // 0 when m == -inf
-        l *= corr;
+      sc[0][u] = x0;
+      sc[1][u] = x1;
+      m[0] = fmaxf(m[0], x0);
+      m[1] = fmaxf(m[1], x1);
+    }
 #pragma unroll
-        for (int c = 0; c < D16; ++c) acc[c] *= corr;
-        m = cm;
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int t = lane + 32 * (kh * 8 + u);
+      const float p0 = m[0] == -INFINITY ? 0.f : sm100::ex2_approx(sc[0][u] - m[0]);  // 0 for -inf
+      const float p1 = m[1] == -INFINITY ? 0.f : sm100::ex2_approx(sc[1][u] - m[1]);
+      l[0] += p0;
+      l[1] += p1;
+      if (t < n) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = lane + 32 * (half * 8 + u);
-        const float pj = sm100::ex2_approx(sc[u] - m);  // 0 for -inf
-        l += pj;
-        if (t < n) {
-#pragma unroll
-          for (int c = 0; c < D16; c += 4) {
-            const float4 v4 = sv[t][(c / 4) ^ ((t >> 1) & 3)];
-            acc[c] = fmaf(pj, v4.x, acc[c]);
-            acc[c + 1] = fmaf(pj, v4.y, acc[c + 1]);
-            acc[c + 2] = fmaf(pj, v4.z, acc[c + 2]);
-            acc[c + 3] = fmaf(pj, v4.w, acc[c + 3]);
-          }
+        for (int c = 0; c < D16; c += 4) {
+          const float4 v4 = sv[t][(c / 4) ^ ((t >> 1) & 3)];
+          acc[0][c] = fmaf(p0, v4.x, acc[0][c]);
+          acc[0][c + 1] = fmaf(p0, v4.y, acc[0][c + 1]);
+          acc[0][c + 2] = fmaf(p0, v4.z, acc[0][c + 2]);
+          acc[0][c + 3] = fmaf(p0, v4.w, acc[0][c + 3]);
+          acc[1][c] = fmaf(p1, v4.x, acc[1][c]);
+          acc[1][c + 1] = fmaf(p1, v4.y, acc[1][c + 1]);
+          acc[1][c + 2] = fmaf(p1, v4.z, acc[1][c + 2]);
+          acc[1][c + 3] = fmaf(p1, v4.w, acc[1][c + 3]);
         }
       }
     }
-    // combine the 32 lanes: max, sum, and the 16 columns by a butterfly
-    // reduce-scatter (lane pair (2k, 2k+1) ends with column bits 4..1 of the lane)
-    float M = m;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w = (m == -INFINITY) ? 0.f : sm100::ex2_approx(m - M);
-    l *= w;
+    for (int r = 0; r < 2; ++r) {
+      // combine the 32 lanes: max, sum, and the 16 columns by a butterfly
+      // reduce-scatter (lane pair (2k, 2k+1) ends with column bits 4..1 of the lane)
+      float M = m[r];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float w = (m[r] == -INFINITY) ? 0.f : sm100::ex2_approx(m[r] - M);
+      float lr = l[r] * w;
 #pragma unroll
-    for (int c = 0; c < D16; ++c) acc[c] *= w;
-    float r8[8], r4[4], r2[2], r1;
+      for (int o = 16; o > 0; o >>= 1) lr += __shfl_xor_sync(0xffffffffu, lr, o);
+      float r8[8], r4[4], r2[2], r1;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const bool hi = lane & 16;
-      r8[k] = (hi ? acc[k + 8] : acc[k]) + __shfl_xor_sync(0xffffffffu, hi ? acc[k] : acc[k + 8], 16);
-    }
+      for (int k = 0; k < 8; ++k) {
+        const bool hi = lane & 16;
+        const float lo_v = acc[r][k] * w, hi_v = acc[r][k + 8] * w;
+        r8[k] = (hi ? hi_v : lo_v) + __shfl_xor_sync(0xffffffffu, hi ? lo_v : hi_v, 16);
+      }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const bool hi = lane & 8;
-      r4[k] = (hi ? r8[k + 4] : r8[k]) + __shfl_xor_sync(0xffffffffu, hi ? r8[k] : r8[k + 4], 8);
-    }
+      for (int k = 0; k < 4; ++k) {
+        const bool hi = lane & 8;
+        r4[k] = (hi ? r8[k + 4] : r8[k]) + __shfl_xor_sync(0xffffffffu, hi ? r8[k] : r8[k + 4], 8);
+      }
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const bool hi = lane & 4;
-      r2[k] = (hi ? r4[k + 2] : r4[k]) + __shfl_xor_sync(0xffffffffu, hi ? r4[k] : r4[k + 2], 4);
-    }
-    {
-      const bool hi = lane & 2;
-      r1 = (hi ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, hi ? r2[0] : r2[1], 2);
-    }
-    r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-    float* pr = part_s + i * kPartStride;
-    if ((lane & 1) == 0) pr[((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = r1;
-    if (lane == 0) {
-      pr[16] = M;
-      pr[17] = l;
+      for (int k = 0; k < 2; ++k) {
+        const bool hi = lane & 4;
+        r2[k] = (hi ? r4[k + 2] : r4[k]) + __shfl_xor_sync(0xffffffffu, hi ? r4[k] : r4[k + 2], 4);
+      }
+      {
+        const bool hi = lane & 2;
+        r1 = (hi ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, hi ? r2[0] : r2[1], 2);
+      }
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      if (r == 1 && !live1) continue;
+      float* pr = part_s + (ir[r] * 2 + kh) * kPartStride;
+      if ((lane & 1) == 0) pr[((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = r1;
+      if (lane == 0) {
+        pr[16] = M;
+        pr[17] = lr;
+      }
     }
   }
-  // every part's partials are in its shared memory; CTA 0 of the cluster
-  // reads them all (distributed shared memory) and writes the rows
+  // every part's partials (two key halves per row) are in its shared memory;
+  // CTA 0 of the cluster reads them all (distributed shared memory) and
+  // writes the rows
   cluster.sync();
   if (part == 0) {
+    const int nslot = 2 * a.ncl;  // (part, half) partials per row
     for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
       float Mk = -INFINITY, lk = 0.f;
-      if (lane < a.ncl) {
-        const float* pr = cluster.map_shared_rank(part_s, lane) + i * kPartStride;
+      if (lane < nslot) {
+        const float* pr = cluster.map_shared_rank(part_s, lane >> 1) + (i * 2 + (lane & 1)) * kPartStride;
         Mk = pr[16];
         lk = pr[17];
       }
@@ -525,11 +541,12 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
       float den = wk * lk;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      // lane c (< 16) sums column c over the parts
+      // lane c (< 16) sums column c over the partials
       float num = 0.f;
-      for (int k = 0; k < a.ncl; ++k) {
+      for (int k = 0; k < nslot; ++k) {
         const float w_k = __shfl_sync(0xffffffffu, wk, k);
-        if (lane < D16 && w_k > 0.f) num = fmaf(w_k, cluster.map_shared_rank(part_s, k)[i * kPartStride + lane], num);
+        if (lane < D16 && w_k > 0.f)
+          num = fmaf(w_k, cluster.map_shared_rank(part_s, k >> 1)[(i * 2 + (k & 1)) * kPartStride + lane], num);
       }
       const float val = den > 0.f ? num / den : 0.f;
       const float nb = __shfl_down_sync(0xffffffffu, val, 1);
@@ -612,7 +629,7 @@ cudaError_t launch_split_kv(const Params& p, cudaStream_t stream) {
     a.p = p;
     a.ncl = kClusterMax;
     a.chunk = (p.Tkv + kClusterMax - 1) / kClusterMax;
-    const size_t smem = (size_t)2 * kClusterChunk * (D16 / 4) * sizeof(float4) + (size_t)kRowsMax * kPartStride * 4;
+    const size_t smem = (size_t)2 * kClusterChunk * (D16 / 4) * sizeof(float4) + (size_t)kRowsMax * 2 * kPartStride * 4;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [&] {
