@@ -14,7 +14,11 @@ import os
 from typing import Optional, Sequence
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsdpa.so")
+RELEASE_LIB_PATH = os.path.join(_PKG, "libsdpa.so")
+# the build with device-side index checks (see sdpa_debug_checks)
+DEBUG_LIB_PATH = os.path.join(_PKG, "libsdpa_debug.so")
+# SDPA_DEBUG=1 in the environment selects the debug build for this process
+LIB_PATH = DEBUG_LIB_PATH if os.environ.get("SDPA_DEBUG", "0") not in ("", "0") else RELEASE_LIB_PATH
 
 SDPA_F32, SDPA_BF16 = 0, 1
 MASK_NONE, MASK_CAUSAL, MASK_SLIDING, MASK_FLOAT, MASK_BOOL = 0, 1, 2, 3, 4
@@ -23,12 +27,12 @@ PATHS = {"auto": PATH_AUTO, "exact": PATH_EXACT, "tcgen05": PATH_TCGEN05,
          "small_d": PATH_SMALL_D, "split_kv": PATH_SPLIT_KV, "tc_persistent": PATH_TC_PERSISTENT}
 STATUS = {0: "SDPA_OK", -1: "SDPA_ERR_INVALID_ARG", -2: "SDPA_ERR_UNSUPPORTED",
           -3: "SDPA_ERR_MISALIGNED", -4: "SDPA_ERR_CUDA", -5: "SDPA_ERR_TIMEOUT",
-          -6: "SDPA_ERR_CAPACITY"}
+          -6: "SDPA_ERR_CAPACITY", -7: "SDPA_ERR_DEVICE_INDEX"}
 
 # Every symbol include/sdpa.h declares.
 EXPORTS = ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_merge", "sdpa_select_path", "sdpa_fwd_host",
-           "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_selftest_wait_timeout", "sdpa_strerror",
-           "sdpa_version")
+           "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_debug_checks", "sdpa_selftest_wait_timeout",
+           "sdpa_selftest_index_check", "sdpa_strerror", "sdpa_version")
 
 
 class SdpaError(RuntimeError):
@@ -56,8 +60,9 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libsdpa.so is not built ({LIB_PATH}); run "
-                              "`python -m attention_sdpa_fwd_b200.build`")
+            flag = " --debug" if LIB_PATH == DEBUG_LIB_PATH else ""
+            raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
+                              f"`python -m attention_sdpa_fwd_b200.build{flag}`")
         L = ctypes.CDLL(LIB_PATH)
         L.sdpa_fwd.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
         L.sdpa_fwd_ex.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
@@ -68,11 +73,13 @@ def lib():
         L.sdpa_fwd_split_kv_static.argtypes = _COMMON + [_f32, _i32, _vp, _vp, _vp]
         L.sdpa_last_device_error.argtypes = [_vp]
         L.sdpa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, _vp]
+        L.sdpa_selftest_index_check.argtypes = [ctypes.c_longlong, ctypes.c_longlong, _vp]
+        L.sdpa_debug_checks.argtypes = []
         L.sdpa_strerror.argtypes = [_i32]
         L.sdpa_strerror.restype = ctypes.c_char_p
         for name in ("sdpa_fwd", "sdpa_fwd_ex", "sdpa_fwd_strided", "sdpa_merge", "sdpa_fwd_host", "sdpa_select_path",
                      "sdpa_fwd_split_kv_static", "sdpa_last_device_error", "sdpa_selftest_wait_timeout",
-                     "sdpa_version"):
+                     "sdpa_selftest_index_check", "sdpa_debug_checks", "sdpa_version"):
             getattr(L, name).restype = _i32
         _lib = L
     return _lib
@@ -140,6 +147,14 @@ def sdpa_selftest_wait_timeout(limit_ns, stream) -> int:
 
 def sdpa_strerror(status: int) -> str:
     return lib().sdpa_strerror(status).decode()
+
+
+def sdpa_selftest_index_check(index, extent, stream) -> int:
+    return lib().sdpa_selftest_index_check(index, extent, stream)
+
+
+def sdpa_debug_checks() -> int:
+    return lib().sdpa_debug_checks()
 
 
 def sdpa_version() -> int:

@@ -533,6 +533,21 @@ extern "C" int sdpa_selftest_wait_timeout(unsigned long long limit_ns, cudaStrea
   return selftest_wait_timeout(limit_ns, err, stream);
 }
 
+extern "C" int sdpa_selftest_index_check(long long index, long long extent, cudaStream_t stream) {
+  if (extent < 0) return SDPA_ERR_INVALID_ARG;
+  int* err = error_word_ptr();
+  if (err == nullptr) return SDPA_ERR_CUDA;
+  return selftest_index_check(index, extent, err, stream);
+}
+
+extern "C" int sdpa_debug_checks(void) {
+#ifdef SDPA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 extern "C" int sdpa_last_device_error(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return SDPA_ERR_CUDA;
   int* w = error_word_ptr();
@@ -543,7 +558,7 @@ extern "C" int sdpa_last_device_error(cudaStream_t stream) {
     const int zero = 0;
     if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SDPA_ERR_CUDA;
     mark_workspace_dirty();  // an abandoned split may have left its counters behind
-    return SDPA_ERR_TIMEOUT;
+    return (host & ERR_INDEX) ? SDPA_ERR_DEVICE_INDEX : SDPA_ERR_TIMEOUT;
   }
   return SDPA_OK;
 }
@@ -557,6 +572,7 @@ extern "C" const char* sdpa_strerror(int status) {
     case SDPA_ERR_CUDA: return "CUDA error";
     case SDPA_ERR_TIMEOUT: return "device-side wait timed out";
     case SDPA_ERR_CAPACITY: return "request exceeds a fixed-size buffer";
+    case SDPA_ERR_DEVICE_INDEX: return "device-side index check failed (debug build)";
   }
   return "unknown status";
 }

@@ -54,7 +54,38 @@ __host__ __device__ __forceinline__ bool strides_multiple_of(const Params& p, lo
   return true;
 }
 
-enum ErrBits { ERR_WAIT_TIMEOUT = 1 };
+enum ErrBits { ERR_WAIT_TIMEOUT = 1, ERR_INDEX = 2 };
+
+// Device-side index checks.  A build compiled with SDPA_DEBUG tests each
+// index a kernel derives (query / key rows, rel-pos table rows, mask and
+// workspace slots, shared-memory slots of the scatter) against its extent
+// before the access; an index outside it sets ERR_INDEX in the error word and
+// the access is skipped (no trap, no fault).  Without SDPA_DEBUG every check
+// is the constant true and compiles away.
+#ifdef SDPA_DEBUG
+__device__ __noinline__ inline void dcheck_fail(int* err) {
+  if (err != nullptr) atomicOr(err, ERR_INDEX);
+}
+__device__ __forceinline__ bool dcheck(int* err, bool ok) {
+  if (!ok) dcheck_fail(err);
+  return ok;
+}
+// 0 <= i < n
+__device__ __forceinline__ bool dcheck_idx(int* err, long long i, long long n) { return dcheck(err, i >= 0 && i < n); }
+// row t of (batch b, query head h): q, out, lse
+__device__ __forceinline__ bool dcheck_q(const Params& p, long long b, long long h, long long t) {
+  return dcheck(p.err, b >= 0 && b < p.B && h >= 0 && h < p.Hq && t >= 0 && t < p.Tq);
+}
+// row t of (batch b, key/value head hk): k, v
+__device__ __forceinline__ bool dcheck_kv(const Params& p, long long b, long long hk, long long t) {
+  return dcheck(p.err, b >= 0 && b < p.B && hk >= 0 && hk < p.Hkv && t >= 0 && t < p.Tkv);
+}
+#else
+__device__ __forceinline__ constexpr bool dcheck(int*, bool) { return true; }
+__device__ __forceinline__ constexpr bool dcheck_idx(int*, long long, long long) { return true; }
+__device__ __forceinline__ constexpr bool dcheck_q(const Params&, long long, long long, long long) { return true; }
+__device__ __forceinline__ constexpr bool dcheck_kv(const Params&, long long, long long, long long) { return true; }
+#endif
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -101,6 +132,8 @@ cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream
 int split_kv_static(const Params& p, sdpa_dtype_t dtype, cudaStream_t stream);
 // One bounded mbarrier wait that runs out (nothing arrives); sets *err.
 int selftest_wait_timeout(unsigned long long limit_ns, int* err, cudaStream_t stream);
+// One index check of i against [0, n) on the device, no memory access at i.
+int selftest_index_check(long long i, long long n, int* err, cudaStream_t stream);
 int num_sms();
 cudaError_t launch_tc(const Params& p, cudaStream_t stream);
 // persistent form of the tensor-core kernel (one CTA per SM over many short problems)

@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
   const int b = blockIdx.z;
   if (i >= p.Tq) return;  // warp-uniform; no block barrier follows
   const int hk = h / p.group;
+  if (!dcheck_q(p, b, h, i)) return;  // debug builds: the row is in q / out
   const int per_warp = D + (p.use_rel ? (p.kh_n + p.kw_n) : 0);
   float* qs = smem + warp * per_warp;
   float* relh = qs + D;
@@ -67,10 +68,14 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     const int qh = (int)(i / p.qw_n), qw = (int)(i % p.qw_n);
     const T* Rh = static_cast<const T*>(p.rel_h);
     const T* Rw = static_cast<const T*>(p.rel_w);
-    for (int a = lane; a < p.kh_n; a += 32)
-      relh[a] = dot_any<T>(qs, Rh + (long long)(qh - a + p.kh_n - 1) * D, D);
-    for (int a = lane; a < p.kw_n; a += 32)
-      relw[a] = dot_any<T>(qs, Rw + (long long)(qw - a + p.kw_n - 1) * D, D);
+    for (int a = lane; a < p.kh_n; a += 32) {
+      const long long r = qh - a + p.kh_n - 1;
+      relh[a] = dcheck_idx(p.err, r, p.qh_n + p.kh_n - 1) ? dot_any<T>(qs, Rh + r * D, D) : 0.f;
+    }
+    for (int a = lane; a < p.kw_n; a += 32) {
+      const long long r = qw - a + p.kw_n - 1;
+      relw[a] = dcheck_idx(p.err, r, p.qw_n + p.kw_n - 1) ? dot_any<T>(qs, Rw + r * D, D) : 0.f;
+    }
     __syncwarp();
   }
 
@@ -93,7 +98,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
   for (long long j0 = lo; j0 < hi; j0 += 32) {
     const long long j = j0 + lane;
     float s = -INFINITY;
-    if (j < hi) {
+    if (j < hi && dcheck_kv(p, b, hk, j)) {
       s = p.scale * (p.k_vec16 ? dot_row<T, D>(qs, kb + j * p.skt) : dot_any<T>(qs, kb + j * p.skt, D));
       if (p.use_rel) s += relh[j / p.kw_n] + relw[j % p.kw_n];
       if (p.mask_kind == SDPA_MASK_ADD_FLOAT) {
@@ -118,7 +123,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     const int nk = (int)((hi - j0) < 32 ? (hi - j0) : 32);
     for (int t = 0; t < nk; ++t) {
       const float pt = __shfl_sync(0xffffffffu, pj, t);
-      if (owns_cols) {
+      if (owns_cols && dcheck_kv(p, b, hk, j0 + t)) {
         const T* vr = vb + (j0 + t) * p.svt + col0;
 #pragma unroll
         for (int c = 0; c < CPL; ++c) acc[c] = fmaf(pt, to_f32(vr[c]), acc[c]);

@@ -368,7 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
     for (int it = 0; it < n_units && ok; ++it) {
       const UnitPos u = unit_pos(args, blockIdx.x + it * G);
       const long long qi = (long long)u.q0 + row;
-      const bool row_valid = qi < args.Tq;
+      // (debug builds: the unit's batch and head lie inside the problem)
+      const bool row_valid = qi < args.Tq && dcheck(args.err, qi >= 0 && u.h >= 0 && u.h < args.Hq &&
+                                                                  ((long long)u.b * args.Hq + u.h) * args.nqblk < args.units);
 
       // this unit's rel_h / rel_w (log2 e prescaled): projections from the P
       // columns into this row's shared-memory slots; rel_w then in registers
@@ -388,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int k = base_idx - i;  // key-grid coordinate reached through table row i
-            if (k >= 0 && k < nk) (w == 0 ? relh_s : relw_s)[k * 256 + row] = __uint_as_float(r[i]) * kLog2e;
+            if (k >= 0 && k < nk && dcheck_idx(args.err, k, w == 0 ? kRelH : KW))
+              (w == 0 ? relh_s : relw_s)[k * 256 + row] = __uint_as_float(r[i]) * kLog2e;
           }
         }
 #pragma unroll

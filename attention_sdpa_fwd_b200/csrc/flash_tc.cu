@@ -202,6 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   const int j_begin = jb + (int)((long long)(je - jb) * sidx / nsplit);
   const int j_end = jb + (int)((long long)(je - jb) * (sidx + 1) / nsplit);
   const int n_tiles = j_end - j_begin;
+  // debug builds: the unit and its share of key tiles lie inside the problem
+  // (uniform over the CTA, so the whole CTA leaves before any barrier)
+  if (!dcheck(args.err, unit >= 0 && (long long)unit < (long long)args.B * args.Hq * args.nqblk && sidx < nsplit &&
+                            j_begin >= 0 && j_begin <= j_end && (long long)j_end * BN < (long long)args.Tkv + BN))
+    return;
 
   if (tid == 0) {
     *abort_flag = 0;
@@ -515,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int k = base_idx - (c0 + i);  // key-grid coordinate reached through table row c0+i
-                if (k >= 0 && k < nk) {
+                if (k >= 0 && k < nk && dcheck_idx(args.err, k, w == 0 ? kRelHMax : KW)) {
                   const float val = __uint_as_float(r[i]) * kLog2e;
                   if (w == 1 && kRwInSmem)
                     // this row's slice, float4 groups XOR-swizzled by row: the
@@ -762,13 +767,14 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       // partial O as [part][D/4][256 rows] float4: one store instruction of a
       // warp writes 512 contiguous bytes
       float4* wso = reinterpret_cast<float4*>(args.ws_o) + (part0 + sidx) * (D / 4) * 256 + row;
+      const bool ws_ok = dcheck_idx(args.err, part0 + sidx, (long long)gridDim.x - args.n_full);
       if (live) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(o_addr + c0, r);
           tmem_wait_ld();
-          if (have) {
+          if (have && ws_ok) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
               __stcg(wso + ((c0 + c) / 4) * 256,
@@ -777,7 +783,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           }
         }
       }
-      __stcg(args.ws_ml + (part0 + sidx) * 256 + row, make_float2(have ? m_run : -INFINITY, have ? l_run : 0.f));
+      if (ws_ok)
+        __stcg(args.ws_ml + (part0 + sidx) * 256 + row, make_float2(have ? m_run : -INFINITY, have ? l_run : 0.f));
       // The barrier orders every thread's stores before thread 0's gpu-scope
       // fence and ticket increment (fences are cumulative); the last arriver's
       // fence after its increment acquires the other parts' stores.

@@ -7,6 +7,12 @@
 // nothing ever arrives on, then returns.  The wait always ends (the limit is
 // checked on the host to be at most 2 s), no memory is touched except the
 // error word, and the CUDA context stays usable.
+//
+// sdpa_selftest_index_check: runs one device-side index check (the checks a
+// build with SDPA_DEBUG compiles into the kernels) on an index and an extent
+// the caller gives.  Nothing is read or written at the index: the kernel only
+// evaluates the check, which in a debug build sets the error word when the
+// index is outside [0, n), and in a release build is the constant true.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -25,7 +31,16 @@ __global__ void wait_timeout_kernel(int* err, unsigned long long limit_ns) {
   }
 }
 
+__global__ void index_check_kernel(int* err, long long i, long long n) {
+  if (threadIdx.x == 0) (void)dcheck_idx(err, i, n);
+}
+
 }  // namespace
+
+int selftest_index_check(long long i, long long n, int* err, cudaStream_t stream) {
+  index_check_kernel<<<1, 32, 0, stream>>>(err, i, n);
+  return cudaGetLastError() == cudaSuccess ? SDPA_OK : SDPA_ERR_CUDA;
+}
 
 int selftest_wait_timeout(unsigned long long limit_ns, int* err, cudaStream_t stream) {
   wait_timeout_kernel<<<1, 32, 0, stream>>>(err, limit_ns);

@@ -90,7 +90,9 @@ typedef enum {
   SDPA_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (launch, copy) */
   SDPA_ERR_TIMEOUT = -5,      /* a device-side bounded wait expired (see
                                  sdpa_last_device_error) */
-  SDPA_ERR_CAPACITY = -6      /* the request exceeds a fixed-size buffer of this entry point */
+  SDPA_ERR_CAPACITY = -6,     /* the request exceeds a fixed-size buffer of this entry point */
+  SDPA_ERR_DEVICE_INDEX = -7  /* debug build only: a kernel's device-side index check failed
+                                 (see sdpa_debug_checks) */
 } sdpa_status;
 
 /* Kernel families.  AUTO picks per shape; the others force one family and
@@ -276,10 +278,32 @@ int sdpa_fwd_split_kv_static(const void* q, const void* k, const void* v, void* 
                              int mask_kind, const void* mask_ptr, float* lse, cudaStream_t stream);
 
 /* Synchronises `stream`, then returns and clears the device error word of the
-   current device: SDPA_OK, or SDPA_ERR_TIMEOUT when a kernel gave up a bounded
-   wait since the last call (its output is then undefined), or SDPA_ERR_CUDA
-   when the synchronisation itself failed. */
+   current device: SDPA_OK; SDPA_ERR_DEVICE_INDEX when, in a debug build, a
+   kernel's index check failed since the last call; SDPA_ERR_TIMEOUT when a
+   kernel gave up a bounded wait since the last call (output undefined in
+   either case); or SDPA_ERR_CUDA when the synchronisation itself failed. */
 int sdpa_last_device_error(cudaStream_t stream);
+
+/* 1 when this library was built with SDPA_DEBUG (libsdpa_debug.so), else 0.
+   A debug build tests every index its kernels derive -- query and key rows,
+   rel-pos table rows (the qh - kh + Kh - 1 and qw - kw + Kw - 1 of the
+   decomposed bias), mask and workspace slots, shared-memory slots of the
+   rel-pos scatter -- against its extent before the access.  A failed check
+   skips the access and sets the device error word, which
+   sdpa_last_device_error reports as SDPA_ERR_DEVICE_INDEX: no trap, fault or
+   hang.  Results of a debug build equal the release build's; only speed
+   differs.  Host-only: needs no GPU. */
+int sdpa_debug_checks(void);
+
+/* Self-test of the device-side index checks (the library's own
+   instrumentation; the pages have no counterpart).  Enqueues on `stream` one
+   kernel whose single thread evaluates the index check of `index` against
+   [0, extent) and touches no memory at `index`.  In a debug build an index
+   outside the extent sets the device error word (the next
+   sdpa_last_device_error returns SDPA_ERR_DEVICE_INDEX); in a release build
+   the check is compiled out and nothing is set.  extent < 0:
+   SDPA_ERR_INVALID_ARG before any launch. */
+int sdpa_selftest_index_check(long long index, long long extent, cudaStream_t stream);
 
 /* Self-test of the failure detection above (the pages have no counterpart;
    it checks this library's own error path).  Enqueues on `stream` one kernel

@@ -39,7 +39,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_version_and_strerror(L):
     assert S.sdpa_version() >= 100
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert S.sdpa_strerror(code) not in ("", "unknown status")
     assert S.sdpa_strerror(12345) == "unknown status"
 

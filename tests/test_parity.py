@@ -67,6 +67,14 @@ CASES = [
        mask_heads=1, seed=44),
     S_("d16_sliding_long_kv", BF16, 1, 2, 2, 16, 3000, 16, mask_kind=W.MASK_SLIDING, window=700, offset=2000,
        seed=45),
+    # head_dim 16, short query axis and enough heads for the small-d kernel to
+    # pack several heads per CTA (16 heads of 7 rows; 4 heads of 30 rows; 2
+    # heads of 16 rows with the second CTA's second group past the last head)
+    S_("d16_packed16_causal_gqa", BF16, 150, 16, 8, 7, 19, 16, mask_kind=W.MASK_CAUSAL, offset=11, seed=46),
+    S_("d16_packed4_float_mask", BF16, 80, 8, 8, 30, 70, 16, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=8, seed=47),
+    S_("d16_packed2_sliding_odd_heads", BF16, 160, 3, 3, 16, 50, 16, mask_kind=W.MASK_SLIDING, window=9,
+       offset=20, seed=48),
     # rel-pos shapes the tensor-core path specialises (key-grid width 14/16/32/64)
     S_("relpos_bf16_d64_12x16", BF16, 2, 3, 3, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5, seed=27),
     S_("relpos_bf16_d64_8x32", BF16, 1, 4, 2, 256, 256, 64, q_hw=(8, 32), k_hw=(8, 32), rel_std=0.5, seed=28),
