@@ -415,17 +415,40 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
   const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, 0);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, 0);
-  for (int t = threadIdx.x; t < n; t += kSplitThreads) {
-    if (!dcheck_kv(p, b, hk, j0 + t)) continue;
-    float f[D16];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt)), f);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt) + 1), f + 8);
+  // stage the part: each thread moves the K and V rows (32 B each) of keys
+  // tid and tid + 256, all eight 16-byte loads issued before the first
+  // conversion
+  static_assert(kClusterChunk == 2 * kSplitThreads, "two keys per thread");
+  {
+    uint4 raw[2][4];
+    bool have[2];
 #pragma unroll
-    for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt)), f);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt) + 1), f + 8);
+    for (int u = 0; u < 2; ++u) {
+      const int t = threadIdx.x + u * kSplitThreads;
+      have[u] = t < n && dcheck_kv(p, b, hk, j0 + t);
+      if (have[u]) {
+        const uint4* kr = reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt);
+        const uint4* vr = reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt);
+        raw[u][0] = __ldg(kr);
+        raw[u][1] = __ldg(kr + 1);
+        raw[u][2] = __ldg(vr);
+        raw[u][3] = __ldg(vr + 1);
+      }
+    }
 #pragma unroll
-    for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+    for (int u = 0; u < 2; ++u) {
+      const int t = threadIdx.x + u * kSplitThreads;
+      if (!have[u]) continue;
+      float f[D16];
+      bf16x8_to_f32(raw[u][0], f);
+      bf16x8_to_f32(raw[u][1], f + 8);
+#pragma unroll
+      for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+      bf16x8_to_f32(raw[u][2], f);
+      bf16x8_to_f32(raw[u][3], f + 8);
+#pragma unroll
+      for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+    }
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -540,12 +563,13 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
     }
   }
   // every part's partials (two key halves per row) are in its shared memory;
-  // CTA 0 of the cluster reads them all (distributed shared memory) and
-  // writes the rows
+  // row i is merged by part i % ncl, which reads the row's partials from all
+  // parts (distributed shared memory) and writes it: the merge of a row of 8
+  // query rows is spread over the whole cluster
   cluster.sync();
-  if (part == 0) {
+  {
     const int nslot = 2 * a.ncl;  // (part, half) partials per row
-    for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
+    for (int i = part + a.ncl * warp; i < p.Tq; i += a.ncl * (kSplitThreads / 32)) {
       float Mk = -INFINITY, lk = 0.f;
       if (lane < nslot) {
         const float* pr = cluster.map_shared_rank(part_s, lane >> 1) + (i * 2 + (lane & 1)) * kPartStride;
@@ -561,9 +585,10 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
       for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
       // lane c (< 16) sums column c over the partials
       float num = 0.f;
-      for (int k = 0; k < nslot; ++k) {
+#pragma unroll
+      for (int k = 0; k < 2 * kClusterMax; ++k) {
         const float w_k = __shfl_sync(0xffffffffu, wk, k);
-        if (lane < D16 && w_k > 0.f)
+        if (k < nslot && lane < D16 && w_k > 0.f)
           num = fmaf(w_k, cluster.map_shared_rank(part_s, k >> 1)[(i * 2 + (k & 1)) * kPartStride + lane], num);
       }
       const float val = den > 0.f ? num / den : 0.f;
@@ -575,7 +600,7 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
       if (lane == 0 && p.lse) p.lse[zq * p.Tq + i] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
     }
   }
-  // keep every part's shared memory alive until CTA 0 has read it
+  // keep every part's shared memory alive until every part has read it
   cluster.sync();
 }
 
