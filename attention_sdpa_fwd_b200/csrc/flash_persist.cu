@@ -69,6 +69,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only whe
 
 struct PsArgs {
   CUtensorMap tq, tk, tv, trh, trw;
+  CUtensorMap to;  // out, 32-row boxes: each softmax warp stores its rows with one TMA store
   void* out;
   long long sob, soh, sot;
   float* lse;
@@ -93,7 +94,7 @@ struct PLayout {
   static constexpr int oRel = oTab + (KW > 0 ? 2 * kTabBytes : 0);
   static constexpr int kRelRows = KW > 0 ? kRelH + KW : 0;  // rel_h rows then rel_w rows, 256 floats each
   static constexpr int oBar = oRel + kRelRows * 256 * 4;
-  static constexpr int kBars = 4 * NS + 15;
+  static constexpr int kBars = 4 * NS + 17;
   static constexpr int kTotal = oBar + kBars * 8 + 16;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
   uint64_t* rel_mma = q_full + 12;    // a unit's rel projections in TMEM (MMA commit, once per unit)
   uint64_t* tab_full = q_full + 13;   // rel tables landed (once)
   uint64_t* fin = q_full + 14;        // last commit before TMEM release
+  uint64_t* o_drained = q_full + 15;  // [2]  the unit's O rows staged in that Q buffer stored (8 arrivals)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + L::kBars);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
 
@@ -156,6 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
     mbar_init(&s_free[1], kRows);
     mbar_init(&p_full[0], kRows);
     mbar_init(&p_full[1], kRows);
+    mbar_init(&o_drained[0], 8);
+    mbar_init(&o_drained[1], 8);
     fence_mbar_init();
     if (n_units > 0) {
       // the first unit's Q, the rel tables and K tile 0 go out before the
@@ -225,14 +229,16 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
     } else if (warp == 10) {
       // ---------------------------------------------------------- Q producer
       // The Q tiles of unit it go into buffer it & 1 once every MMA of unit
-      // it - 2 is done (a warp of its own, so that waiting for that never
-      // holds back the K/V stream).
+      // it - 2 is done and the output rows unit it - 2 staged there are
+      // stored (a warp of its own, so that waiting for that never holds back
+      // the K/V stream).
       if (lane == 0 && n_units > 1) {
         bool ok = true;
         int q_issued = 1;
         for (int it = 1; it < n_units && ok; ++it) {
           const int qb = it & 1;
           if (it >= 2) ok = mbar_wait(&q_empty[qb], ((it >> 1) - 1) & 1, abort_v, args.err);
+          if (ok && it >= 2) ok = mbar_wait(&o_drained[qb], ((it >> 1) - 1) & 1, abort_v, args.err);
           if (!ok) break;
           const UnitPos u = unit_pos(args, blockIdx.x + it * G);
           mbar_expect_tx(&q_full[qb], 2 * L::kQBytes);
@@ -481,13 +487,26 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
       }
       if (!ok) break;
 
-      // epilogue: O / l -> bf16 (rows past Tq are not stored)
+      // epilogue: O / l -> bf16 rows staged in this unit's Q tile t (its last
+      // Q.K^T, which this warp waited for, was the tile's last reader), then
+      // one TMA store of the warp's 32 rows (rows past Tq are not written);
+      // the Q loader refills the buffer once every warp's store has read it
       ok = __all_sync(0xffffffffu, mbar_wait(&o_ready[t], (it * nt + nt - 1) & 1, abort_v, args.err));
       if (!ok) break;
       tc_fence_after();
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(args.out) + (long long)u.b * args.sob +
-                            (long long)u.h * args.soh + qi * args.sot;
-      tile::store_o_row<kD>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, orow, row_valid);
+      uint8_t* stage = sQ + (it & 1) * L::kQBuf + t * L::kQBytes + (warp & 3) * 32 * 128;
+      tile::stage_o_row_sw128<kD>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, stage + lane * 128, lane);
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        const int r0 = u.q0 + t * kRows + (warp & 3) * 32;
+        if (r0 < args.Tq) {
+          tma_store_4d(&args.to, stage, 0, r0, u.h, u.b);
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+        mbar_arrive(&o_drained[it & 1]);
+      }
       if (row_valid && args.lse)
         args.lse[((long long)u.b * args.Hq + u.h) * args.Tq + qi] =
             l_run > 0.f ? m_run * kLn2 + logf(l_run) : -INFINITY;
@@ -572,6 +591,7 @@ cudaError_t launch_tc_persist(const Params& p, cudaStream_t stream) {
   bool ok = make_tmap_4d(&a.tq, p.q, bf, p.d, p.Tq, p.Hq, p.B, 2 * p.sqt, 2 * p.sqh, 2 * p.sqb, 64, kRows, true);
   ok = ok && make_tmap_4d(&a.tk, p.k, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.skt, 2 * p.skh, 2 * p.skb, 64, BN, true);
   ok = ok && make_tmap_4d(&a.tv, p.v, bf, p.d, p.Tkv, p.Hkv, p.B, 2 * p.svt, 2 * p.svh, 2 * p.svb, 64, BN, true);
+  ok = ok && make_tmap_4d(&a.to, p.out, bf, p.d, p.Tq, p.Hq, p.B, 2 * p.sot, 2 * p.soh, 2 * p.sob, 64, 32, true);
   if (p.use_rel) {
     // 32-row boxes (Qh + Kh - 1 <= 32 table rows); rows past a table read as zero
     const uint64_t nh = p.qh_n + p.kh_n - 1, nw = p.qw_n + p.kw_n - 1;

@@ -107,5 +107,30 @@ __device__ __forceinline__ void store_o_row(uint32_t o_addr, float inv, __nv_bfl
   }
 }
 
+// The same epilogue into shared memory for a TMA store: the row's 64 bf16
+// values (128 bytes) at srow in the 128-byte swizzle of a tensor map with
+// 128-byte rows -- 16-byte piece c at position c ^ (r & 7), r the row's index
+// in its 1024-byte-aligned block (so a warp's 32 rows hit every bank group).
+template <int D>
+__device__ __forceinline__ void stage_o_row_sw128(uint32_t o_addr, float inv, uint8_t* srow, int r) {
+  static_assert(D == 64, "one 128-byte row");
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(o_addr + c0, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 32; c += 8) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(v[c + 0]) * inv, __uint_as_float(v[c + 1]) * inv);
+      w.y = pack_bf16x2(__uint_as_float(v[c + 2]) * inv, __uint_as_float(v[c + 3]) * inv);
+      w.z = pack_bf16x2(__uint_as_float(v[c + 4]) * inv, __uint_as_float(v[c + 5]) * inv);
+      w.w = pack_bf16x2(__uint_as_float(v[c + 6]) * inv, __uint_as_float(v[c + 7]) * inv);
+      const int piece = (c0 + c) >> 3;
+      *reinterpret_cast<uint4*>(srow + ((piece ^ (r & 7)) << 4)) = w;
+    }
+  }
+}
+
 }  // namespace tile
 }  // namespace sdpa
