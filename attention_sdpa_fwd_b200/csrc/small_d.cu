@@ -382,17 +382,75 @@ __global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a)
   if (threadIdx.x == 0) a.ws_cnt[zq] = 0;  // ready for the next launch
 }
 
+// ------------------------------------------------------------------ tensor-core fragments
+// mma.sync m16n8k16, bf16 operands, fp32 accumulate.  Thread (g, t) =
+// (lane / 4, lane % 4) of a warp holds: of a 16x16 A tile, rows g and g + 8 at
+// columns 2t, 2t + 1 (registers 0, 1) and 2t + 8, 2t + 9 (registers 2, 3); of
+// a 16x8 B tile, column g at rows 2t, 2t + 1 (register 0) and 2t + 8, 2t + 9
+// (register 1); of the 16x8 fp32 accumulator, rows g (c0, c1) and g + 8
+// (c2, c3) at columns 2t, 2t + 1.  The S = Q K^T accumulators of two 8-key
+// tiles, packed to bf16, are exactly the A operand of O += P V over those 16
+// keys, so P never leaves registers.  Operands come from shared memory
+// through ldmatrix.
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+               "{%8, %9}, {%0, %1, %2, %3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Byte offset of 16-byte half h (d 0..7 or 8..15) of row r in a [rows][16]
+// bf16 array: halves swap every 4 rows, so the 8 rows one ldmatrix matrix
+// reads hit all 32 banks once.
+__device__ __forceinline__ uint32_t sw32(int r, int h) { return (uint32_t)(r * 32 + ((h ^ ((r >> 2) & 1)) << 4)); }
+
+// The A operand (rows row0 .. row0 + 15) of a [rows][16] bf16 array at base.
+__device__ __forceinline__ void ldsm_a(uint32_t (&a)[4], uint32_t base, int row0, int lane) {
+  ldsm_x4(a, base + sw32(row0 + (lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4));
+}
+// K of keys key0 .. key0 + 15 as the B operands of two 8-key tiles of S = Q K^T:
+// r[0], r[1] for keys key0 .. + 7, r[2], r[3] for keys key0 + 8 .. + 15.
+__device__ __forceinline__ void ldsm_k(uint32_t (&r)[4], uint32_t base, int key0, int lane) {
+  ldsm_x4(r, base + sw32(key0 + (lane & 7) + (lane >> 4) * 8, (lane >> 3) & 1));
+}
+// V of keys key0 .. key0 + 15 as the B operands of O += P V: r[0], r[1] for
+// value columns 0 .. 7, r[2], r[3] for columns 8 .. 15.
+__device__ __forceinline__ void ldsm_v(uint32_t (&r)[4], uint32_t base, int key0, int lane) {
+  ldsm_x4_t(r, base + sw32(key0 + (lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4));
+}
+
 // ------------------------------------------------------------------ split_kv over a cluster
 // The same split of the key axis, with the parts of one (batch, head) in one
 // thread-block cluster: each CTA leaves its partial (O, m, l) per query row
-// in its own shared memory, and CTA 0 of the cluster merges them through
-// distributed shared memory -- no global workspace, fence or ticket, so the
-// whole forward is one pass over K and V.  Used when the key axis fits in 8
-// parts of at most 512 keys.
+// in its own shared memory, and the parts merge through distributed shared
+// memory -- no global workspace, fence or ticket, so the whole forward is one
+// pass over K and V.  Used when the key axis fits in 8 parts of at most 512
+// keys.  Inside a part, K and V are staged as bf16 with 16-byte loads (two
+// keys per thread), and warp w takes 64 of the keys: for every 16-row tile of
+// query rows, S = Q K^T, the softmax over its 64 keys and O = P V run on the
+// tensor cores (mma.sync).  The warps' partials merge in the CTA, the CTAs'
+// through the cluster.
 constexpr int kClusterMax = 8;      // portable cluster size
 constexpr int kClusterChunk = 512;  // keys per CTA (at most)
-constexpr int kRowsMax = 64;        // query rows the partial area holds
+constexpr int kWarpKeys = kClusterChunk / (kSplitThreads / 32);  // 64 keys per warp
+constexpr int kRowsMax = 64;        // query rows the partial areas hold
 constexpr int kPartStride = 20;     // floats per row partial: 16 O, m, l, pad
+// dynamic shared memory: K and V (bf16 rows), Q rows, the warps' partials,
+// the CTA's partials
+constexpr int kClK = 0, kClV = kClusterChunk * 32, kClQ = 2 * kClusterChunk * 32;
+constexpr int kClWarp = kClQ + kRowsMax * 32;
+constexpr int kClPart = kClWarp + (kSplitThreads / 32) * kRowsMax * kPartStride * 4;
+constexpr int kClBytes = kClPart + kRowsMax * kPartStride * 4;
 
 struct ClusterArgs {
   Params p;
@@ -403,202 +461,198 @@ struct ClusterArgs {
 __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(ClusterArgs a) {
   namespace cg = cooperative_groups;
   const Params& p = a.p;
-  extern __shared__ float4 cl_smem[];
-  float4 (*sk)[D16 / 4] = reinterpret_cast<float4 (*)[D16 / 4]>(cl_smem);
-  float4 (*sv)[D16 / 4] = reinterpret_cast<float4 (*)[D16 / 4]>(cl_smem + kClusterChunk * (D16 / 4));
-  float* part_s = reinterpret_cast<float*>(cl_smem + 2 * kClusterChunk * (D16 / 4));  // [Tq][2 halves][kPartStride]
+  constexpr int kWarps = kSplitThreads / 32;
+  extern __shared__ __align__(128) uint8_t cl_smem[];
+  float* warp_s = reinterpret_cast<float*>(cl_smem + kClWarp);  // [kWarps][kRowsMax][kPartStride]
+  float* part_s = reinterpret_cast<float*>(cl_smem + kClPart);  // [kRowsMax][kPartStride], read by the cluster
+  const uint32_t k_s = sm100::smem_u32(cl_smem + kClK), v_s = sm100::smem_u32(cl_smem + kClV);
+  const uint32_t q_s = sm100::smem_u32(cl_smem + kClQ);
   cg::cluster_group cluster = cg::this_cluster();
   const int part = (int)cluster.block_rank(), h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.group;
   const long long zq = (long long)b * p.Hq + h;
   const long long j0 = (long long)part * a.chunk;
   const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, 0);
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, 0);
-  // stage the part: each thread moves the K and V rows (32 B each) of keys
-  // tid and tid + 256, all eight 16-byte loads issued before the first
-  // conversion
-  static_assert(kClusterChunk == 2 * kSplitThreads, "two keys per thread");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int mrows = (p.Tq + 15) & ~15;  // query rows rounded up to whole 16-row tiles
   {
-    uint4 raw[2][4];
-    bool have[2];
+    // stage K and V rows tid and tid + 256 (zeros past the part) and Q rows
+    // (zeros past Tq), all loads issued before the first store
+    static_assert(kClusterChunk == 2 * kSplitThreads, "two keys per thread");
+    uint4 kv[2][4], qv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int t = threadIdx.x + u * kSplitThreads;
-      have[u] = t < n && dcheck_kv(p, b, hk, j0 + t);
-      if (have[u]) {
-        const uint4* kr = reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt);
-        const uint4* vr = reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt);
-        raw[u][0] = __ldg(kr);
-        raw[u][1] = __ldg(kr + 1);
-        raw[u][2] = __ldg(vr);
-        raw[u][3] = __ldg(vr + 1);
+      const int tk = tid + u * kSplitThreads;
+      kv[u][0] = kv[u][1] = kv[u][2] = kv[u][3] = make_uint4(0, 0, 0, 0);
+      if (tk < n && dcheck_kv(p, b, hk, j0 + tk)) {
+        const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, j0 + tk));
+        const uint4* vr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, j0 + tk));
+        kv[u][0] = __ldg(kr);
+        kv[u][1] = __ldg(kr + 1);
+        kv[u][2] = __ldg(vr);
+        kv[u][3] = __ldg(vr + 1);
       }
+    }
+    if (tid < mrows && tid < p.Tq && dcheck_q(p, b, h, tid)) {
+      const uint4* qr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, tid));
+      qv[0] = __ldg(qr);
+      qv[1] = __ldg(qr + 1);
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int t = threadIdx.x + u * kSplitThreads;
-      if (!have[u]) continue;
-      float f[D16];
-      bf16x8_to_f32(raw[u][0], f);
-      bf16x8_to_f32(raw[u][1], f + 8);
-#pragma unroll
-      for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
-      bf16x8_to_f32(raw[u][2], f);
-      bf16x8_to_f32(raw[u][3], f + 8);
-#pragma unroll
-      for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+      const int tk = tid + u * kSplitThreads;
+      *reinterpret_cast<uint4*>(cl_smem + kClK + sw32(tk, 0)) = kv[u][0];
+      *reinterpret_cast<uint4*>(cl_smem + kClK + sw32(tk, 1)) = kv[u][1];
+      *reinterpret_cast<uint4*>(cl_smem + kClV + sw32(tk, 0)) = kv[u][2];
+      *reinterpret_cast<uint4*>(cl_smem + kClV + sw32(tk, 1)) = kv[u][3];
+    }
+    if (tid < mrows) {
+      *reinterpret_cast<uint4*>(cl_smem + kClQ + sw32(tid, 0)) = qv[0];
+      *reinterpret_cast<uint4*>(cl_smem + kClQ + sw32(tid, 1)) = qv[1];
     }
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl = p.scale * kLog2e;
-  // Warp w takes two query rows, 2 (w & 3) + 8 r and the next, over one half
-  // of the part's keys (w >> 2): every K and V row read from shared memory
-  // serves two query rows, and each row's two key halves become two partials.
-  const int kh = warp >> 2;
-  for (int i0 = 2 * (warp & 3); i0 < p.Tq; i0 += 8) {
-    const int ir[2] = {i0, min(i0 + 1, p.Tq - 1)};
-    const bool live1 = i0 + 1 < p.Tq;
-    float q[2][D16];
-    long long mrow[2];
+  const int kw0 = warp * kWarpKeys;  // this warp's keys within the part: [kw0, kw0 + 64)
+  float* wp = warp_s + warp * kRowsMax * kPartStride;
+  for (int row0 = 0; row0 < p.Tq; row0 += 16) {
+    uint32_t qa[4];
+    ldsm_a(qa, q_s, row0, lane);
+    float x[kWarpKeys / 16][2][4];
+#pragma unroll
+    for (int c = 0; c < kWarpKeys / 16; ++c) {
+      uint32_t kf[4];
+      ldsm_k(kf, k_s, kw0 + 16 * c, lane);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        x[c][u][0] = x[c][u][1] = x[c][u][2] = x[c][u][3] = 0.f;
+        mma16816(x[c][u], qa, kf[2 * u], kf[2 * u + 1]);
+      }
+    }
+    // scores in log2 units with the mask; keys past the part and rows past
+    // Tq score -inf
+    const long long mrow_base = (long long)b * p.msb + (long long)h * p.msh;
+#pragma unroll
+    for (int c = 0; c < kWarpKeys / 16; ++c)
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = row0 + g + (e >> 1) * 8;
+          const int kk = kw0 + 16 * c + 8 * u + 2 * t + (e & 1);
+          float v = x[c][u][e] * sl;
+          if (kk >= n || row >= p.Tq)
+            v = -INFINITY;
+          else
+            v += mask_term(p, mrow_base + (long long)row * p.msq, row, j0 + kk);
+          x[c][u][e] = v;
+        }
+    float mr[2], lr[2] = {0.f, 0.f}, o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, ir[r]);
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q[r]);
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q[r] + 8);
-      mrow[r] = (long long)b * p.msb + (long long)h * p.msh + (long long)ir[r] * p.msq;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kWarpKeys / 16; ++c)
+        mx = fmaxf(mx, fmaxf(fmaxf(x[c][0][2 * r], x[c][0][2 * r + 1]), fmaxf(x[c][1][2 * r], x[c][1][2 * r + 1])));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mr[r] = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     }
-    // this lane's eight keys of the half (lane + 32 u): scores of both rows,
-    // their maxima, then the sums
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, acc[2][D16];
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int c = 0; c < kWarpKeys / 16; ++c) {
+      uint32_t pa[4];
 #pragma unroll
-      for (int c = 0; c < D16; ++c) acc[r][c] = 0.f;
-    float sc[2][8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int t = lane + 32 * (kh * 8 + u);
-      float x0 = -INFINITY, x1 = -INFINITY;
-      if (t < n) {
-        x0 = 0.f;
-        x1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < D16; c += 4) {
-          const float4 k4 = sk[t][(c / 4) ^ ((t >> 1) & 3)];
-          x0 = fmaf(q[0][c], k4.x, fmaf(q[0][c + 1], k4.y, fmaf(q[0][c + 2], k4.z, fmaf(q[0][c + 3], k4.w, x0))));
-          x1 = fmaf(q[1][c], k4.x, fmaf(q[1][c + 1], k4.y, fmaf(q[1][c + 2], k4.z, fmaf(q[1][c + 3], k4.w, x1))));
-        }
-        x0 = x0 * sl + mask_term(p, mrow[0], ir[0], j0 + t);
-        x1 = x1 * sl + mask_term(p, mrow[1], ir[1], j0 + t);
+      for (int r = 0; r < 2; ++r) {
+        const float mu = mr[r] == -INFINITY ? 0.f : mr[r];  // nothing visible: every p is 0
+        const float p00 = sm100::ex2_approx(x[c][0][2 * r] - mu), p01 = sm100::ex2_approx(x[c][0][2 * r + 1] - mu);
+        const float p10 = sm100::ex2_approx(x[c][1][2 * r] - mu), p11 = sm100::ex2_approx(x[c][1][2 * r + 1] - mu);
+        lr[r] += (p00 + p01) + (p10 + p11);
+        pa[r] = pack2(p00, p01);      // keys 2t, 2t + 1 of the 16
+        pa[r + 2] = pack2(p10, p11);  // keys 8 + 2t, 9 + 2t
       }
-      sc[0][u] = x0;
-      sc[1][u] = x1;
-      m[0] = fmaxf(m[0], x0);
-      m[1] = fmaxf(m[1], x1);
+      uint32_t vf[4];
+      ldsm_v(vf, v_s, kw0 + 16 * c, lane);
+      mma16816(o[0], pa, vf[0], vf[1]);
+      mma16816(o[1], pa, vf[2], vf[3]);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int t = lane + 32 * (kh * 8 + u);
-      const float p0 = m[0] == -INFINITY ? 0.f : sm100::ex2_approx(sc[0][u] - m[0]);  // 0 for -inf
-      const float p1 = m[1] == -INFINITY ? 0.f : sm100::ex2_approx(sc[1][u] - m[1]);
-      l[0] += p0;
-      l[1] += p1;
-      if (t < n) {
-#pragma unroll
-        for (int c = 0; c < D16; c += 4) {
-          const float4 v4 = sv[t][(c / 4) ^ ((t >> 1) & 3)];
-          acc[0][c] = fmaf(p0, v4.x, acc[0][c]);
-          acc[0][c + 1] = fmaf(p0, v4.y, acc[0][c + 1]);
-          acc[0][c + 2] = fmaf(p0, v4.z, acc[0][c + 2]);
-          acc[0][c + 3] = fmaf(p0, v4.w, acc[0][c + 3]);
-          acc[1][c] = fmaf(p1, v4.x, acc[1][c]);
-          acc[1][c + 1] = fmaf(p1, v4.y, acc[1][c + 1]);
-          acc[1][c + 2] = fmaf(p1, v4.z, acc[1][c + 2]);
-          acc[1][c + 3] = fmaf(p1, v4.w, acc[1][c + 3]);
-        }
-      }
-    }
+    // this warp's partial of rows row0 + g and row0 + g + 8 (O unnormalised, m, l)
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      // combine the 32 lanes: max, sum, and the 16 columns by a butterfly
-      // reduce-scatter (lane pair (2k, 2k+1) ends with column bits 4..1 of the lane)
-      float M = m[r];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      const float w = (m[r] == -INFINITY) ? 0.f : sm100::ex2_approx(m[r] - M);
-      float lr = l[r] * w;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) lr += __shfl_xor_sync(0xffffffffu, lr, o);
-      float r8[8], r4[4], r2[2], r1;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const bool hi = lane & 16;
-        const float lo_v = acc[r][k] * w, hi_v = acc[r][k + 8] * w;
-        r8[k] = (hi ? hi_v : lo_v) + __shfl_xor_sync(0xffffffffu, hi ? lo_v : hi_v, 16);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const bool hi = lane & 8;
-        r4[k] = (hi ? r8[k + 4] : r8[k]) + __shfl_xor_sync(0xffffffffu, hi ? r8[k] : r8[k + 4], 8);
-      }
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const bool hi = lane & 4;
-        r2[k] = (hi ? r4[k + 2] : r4[k]) + __shfl_xor_sync(0xffffffffu, hi ? r4[k] : r4[k + 2], 4);
-      }
-      {
-        const bool hi = lane & 2;
-        r1 = (hi ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, hi ? r2[0] : r2[1], 2);
-      }
-      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-      if ((r == 1 && !live1) || !dcheck_idx(p.err, ir[r], kRowsMax)) continue;
-      float* pr = part_s + (ir[r] * 2 + kh) * kPartStride;
-      if ((lane & 1) == 0) pr[((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)] = r1;
-      if (lane == 0) {
-        pr[16] = M;
-        pr[17] = lr;
+      const int row = row0 + g + 8 * r;
+      float L = lr[r];
+      L += __shfl_xor_sync(0xffffffffu, L, 1);
+      L += __shfl_xor_sync(0xffffffffu, L, 2);
+      if (row >= p.Tq || !dcheck_idx(p.err, row, kRowsMax)) continue;
+      float* pr = wp + row * kPartStride;
+      pr[2 * t] = o[0][2 * r];
+      pr[2 * t + 1] = o[0][2 * r + 1];
+      pr[8 + 2 * t] = o[1][2 * r];
+      pr[9 + 2 * t] = o[1][2 * r + 1];
+      if (t == 0) {
+        pr[16] = mr[r];
+        pr[17] = L;
       }
     }
   }
-  // every part's partials (two key halves per row) are in its shared memory;
-  // row i is merged by part i % ncl, which reads the row's partials from all
-  // parts (distributed shared memory) and writes it: the merge of a row of 8
-  // query rows is spread over the whole cluster
-  cluster.sync();
-  {
-    const int nslot = 2 * a.ncl;  // (part, half) partials per row
-    for (int i = part + a.ncl * warp; i < p.Tq; i += a.ncl * (kSplitThreads / 32)) {
-      float Mk = -INFINITY, lk = 0.f;
-      if (lane < nslot) {
-        const float* pr = cluster.map_shared_rank(part_s, lane >> 1) + (i * 2 + (lane & 1)) * kPartStride;
-        Mk = pr[16];
-        lk = pr[17];
-      }
-      float M = lk > 0.f ? Mk : -INFINITY;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      const float wk = (lk > 0.f) ? sm100::ex2_approx(Mk - M) : 0.f;
-      float den = wk * lk;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      // lane c (< 16) sums column c over the partials
-      float num = 0.f;
-#pragma unroll
-      for (int k = 0; k < 2 * kClusterMax; ++k) {
-        const float w_k = __shfl_sync(0xffffffffu, wk, k);
-        if (k < nslot && lane < D16 && w_k > 0.f)
-          num = fmaf(w_k, cluster.map_shared_rank(part_s, k >> 1)[(i * 2 + (k & 1)) * kPartStride + lane], num);
-      }
-      const float val = den > 0.f ? num / den : 0.f;
-      const float nb = __shfl_down_sync(0xffffffffu, val, 1);
-      if (lane < D16 && (lane & 1) == 0 && dcheck_q(p, b, h, i)) {
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + o_off(p, b, h, i);
-        *reinterpret_cast<uint32_t*>(orow + lane) = pack2(val, nb);
-      }
-      if (lane == 0 && p.lse) p.lse[zq * p.Tq + i] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
+  __syncthreads();
+  // the CTA's partial of row i from its warps' (warp i % 8 combines row i)
+  for (int i = warp; i < p.Tq; i += kWarps) {
+    float Mk = -INFINITY, lk = 0.f;
+    if (lane < kWarps) {
+      Mk = warp_s[(lane * kRowsMax + i) * kPartStride + 16];
+      lk = warp_s[(lane * kRowsMax + i) * kPartStride + 17];
     }
+    float M = lk > 0.f ? Mk : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wk = lk > 0.f ? sm100::ex2_approx(Mk - M) : 0.f;
+    float den = wk * lk;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    float num = 0.f;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k) {
+      const float w_k = __shfl_sync(0xffffffffu, wk, k);
+      if (lane < D16 && w_k > 0.f) num = fmaf(w_k, warp_s[(k * kRowsMax + i) * kPartStride + lane], num);
+    }
+    if (lane < D16) part_s[i * kPartStride + lane] = num;
+    if (lane == 0) {
+      part_s[i * kPartStride + 16] = M;
+      part_s[i * kPartStride + 17] = den;
+    }
+  }
+  // every part's partials are in its shared memory; row i is merged by part
+  // i % ncl, which reads the row's partials from all parts (distributed
+  // shared memory) and writes it: the merge is spread over the whole cluster
+  cluster.sync();
+  for (int i = part + a.ncl * warp; i < p.Tq; i += a.ncl * kWarps) {
+    float Mk = -INFINITY, lk = 0.f;
+    if (lane < a.ncl) {
+      const float* pr = cluster.map_shared_rank(part_s, lane) + i * kPartStride;
+      Mk = pr[16];
+      lk = pr[17];
+    }
+    float M = lk > 0.f ? Mk : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wk = (lk > 0.f) ? sm100::ex2_approx(Mk - M) : 0.f;
+    float den = wk * lk;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    // lane c (< 16) sums column c over the parts
+    float num = 0.f;
+#pragma unroll
+    for (int k = 0; k < kClusterMax; ++k) {
+      const float w_k = __shfl_sync(0xffffffffu, wk, k);
+      if (k < a.ncl && lane < D16 && w_k > 0.f)
+        num = fmaf(w_k, cluster.map_shared_rank(part_s, k)[i * kPartStride + lane], num);
+    }
+    const float val = den > 0.f ? num / den : 0.f;
+    const float nb = __shfl_down_sync(0xffffffffu, val, 1);
+    if (lane < D16 && (lane & 1) == 0 && dcheck_q(p, b, h, i)) {
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + o_off(p, b, h, i);
+      *reinterpret_cast<uint32_t*>(orow + lane) = pack2(val, nb);
+    }
+    if (lane == 0 && p.lse) p.lse[zq * p.Tq + i] = den > 0.f ? M * kLn2 + logf(den) : -INFINITY;
   }
   // keep every part's shared memory alive until every part has read it
   cluster.sync();
@@ -688,7 +742,7 @@ cudaError_t launch_split_kv(const Params& p, cudaStream_t stream) {
     a.p = p;
     a.ncl = kClusterMax;
     a.chunk = (p.Tkv + kClusterMax - 1) / kClusterMax;
-    const size_t smem = (size_t)2 * kClusterChunk * (D16 / 4) * sizeof(float4) + (size_t)kRowsMax * 2 * kPartStride * 4;
+    const size_t smem = (size_t)kClBytes;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [&] {
