@@ -61,10 +61,14 @@ constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-po
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3 };
+// TC_FLOAT_TMA: the additive bf16 mask of TC_FLOAT, 64-key tiles brought into
+// shared memory by the producer warp (TMA, two stages per query tile) instead
+// of per-row global loads in the softmax warps.
+enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3, TC_FLOAT_TMA = 4 };
 
 struct TcArgs {
   CUtensorMap tq, tk, tv, trh, trw;
+  CUtensorMap tm;  // TC_FLOAT_TMA: the mask as (key, query row, head, batch), 64 x 128 boxes
   void* out;
   long long sob, soh, sot;  // element strides of out (batch, head, token)
   float* lse;
@@ -92,7 +96,7 @@ struct TcArgs {
   int* err;
 };
 
-template <int D, int BN, int KW, int NS>
+template <int D, int BN, int KW, int NS, bool MT = false>
 struct Layout {
   static constexpr int kPanels = D / 64;
   static constexpr int kQBytes = kPanels * kRowsPerTile * 128;  // one Q tile
@@ -102,8 +106,10 @@ struct Layout {
   static constexpr int oK = oQ + 2 * kQBytes;
   static constexpr int oV = oK + NS * kKVBytes;
   static constexpr int oRel = oV + NS * kKVBytes;
-  static constexpr int oBar = oRel + kRelRows * 256 * 4;
-  static constexpr int kBars = 4 * NS + 20;
+  static constexpr int kMaskBytes = MT ? kRowsPerTile * BN * 2 : 0;  // one query tile's mask tile (bf16)
+  static constexpr int oMask = oRel + kRelRows * 256 * 4;            // [query tile][stage]
+  static constexpr int oBar = oMask + 4 * kMaskBytes;
+  static constexpr int kBars = 4 * NS + 20 + (MT ? 8 : 0);
   static constexpr int kTotal = oBar + kBars * 8 + 32;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -116,7 +122,9 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 
 template <int D, int BN, int KW, int MASK, int NS>
 __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constant__ TcArgs args) {
-  using L = Layout<D, BN, KW, NS>;
+  constexpr bool kMaskTma = (MASK == TC_FLOAT_TMA);
+  static_assert(!kMaskTma || (BN == 64 && KW == 0), "TMA mask tiles: 64 keys of 128-byte rows");
+  using L = Layout<D, BN, KW, NS, kMaskTma>;
   // head_dim 64 leaves 128 TMEM columns free: P_A [384,448), P_B [448,512) get
   // their own columns, so S_t(j+1) = Q_t.K_{j+1}^T can be issued as soon as
   // softmax t has read S_t(j), before P_t(j) exists.  At head_dim 128, P_t
@@ -161,6 +169,11 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   // of its waiter
   uint64_t* s_odd = q_full + 16;         // [2]
   uint64_t* p_odd = q_full + 18;         // [2]   (128 arrivals)
+  // kMaskTma: mask tile of query tile t, stage s at [2 t + s]: TMA -> softmax t,
+  // and softmax t (128 arrivals) -> producer
+  uint64_t* m_full = q_full + 20;        // [4]
+  uint64_t* m_empty = q_full + 24;       // [4]
+  uint8_t* sMask = smem + L::oMask;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + L::kBars);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
 
@@ -218,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     mbar_init(&s_free[1], kRowsPerTile);
     mbar_init(&p_odd[0], kRowsPerTile);
     mbar_init(&p_odd[1], kRowsPerTile);
+    if constexpr (kMaskTma)
+      for (int i = 0; i < 4; ++i) mbar_init(&m_empty[i], kRowsPerTile);
     fence_mbar_init();
     if (n_tiles > 0) {
       // Q (and the rel tables) and the first K tile go out before the TMEM
@@ -299,14 +314,35 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           tma_load_4d(sV + s * L::kKVBytes + p * BN * 128, &args.tv, &v_full[s], p * 64, key0, hk, b);
         v_issued = jj + 1;
       };
+      // kMaskTma: both query tiles' mask tiles of key tile jj, in stage jj & 1
+      int m_issued = 0;
+      auto load_m = [&](int jj) {
+        if constexpr (kMaskTma) {
+          const int s = jj & 1, use = jj >> 1;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (use > 0) ok = mbar_wait(&m_empty[2 * t + s], (use - 1) & 1, abort_v, args.err);
+            if (!ok) return;
+            mbar_expect_tx(&m_full[2 * t + s], L::kMaskBytes);
+            tma_load_4d(sMask + (2 * t + s) * L::kMaskBytes, &args.tm, &m_full[2 * t + s], (j_begin + jj) * BN,
+                        q0 + t * kRowsPerTile, args.msh ? h : 0, args.msb ? b : 0);
+          }
+          m_issued = jj + 1;
+        }
+      };
+      if constexpr (kMaskTma) tma_prefetch_desc(&args.tm);
+      load_m(0);
       constexpr int kAhead = kSDB ? 2 : 1;  // K tiles loaded ahead of V (the MMA issues S two tiles ahead in kSDB)
       for (int jj = 1; jj < n_tiles && ok; ++jj) {
         load_k(jj);
         if (ok && jj >= kAhead) load_v(jj - kAhead);
+        if (ok) load_m(jj);
       }
       for (int jv = max(0, n_tiles - kAhead); jv < n_tiles && ok; ++jv) load_v(jv);
       if (!ok) {
         // abandoned: let the copies already in flight land before the CTA exits
+        if constexpr (kMaskTma)
+          for (int jj = max(0, m_issued - 2); jj < m_issued; ++jj)
+            for (int t = 0; t < 2; ++t) mbar_wait(&m_full[2 * t + (jj & 1)], (jj >> 1) & 1, nullptr, args.err);
         mbar_wait(q_full, 0, nullptr, args.err);
         for (int jj = max(0, k_issued - NS); jj < k_issued; ++jj)
           mbar_wait(&k_full[jj % NS], (jj / NS) & 1, nullptr, args.err);
@@ -663,6 +699,24 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
             }
           }
         }
+      } else if constexpr (kMaskTma) {
+        // this row of the tile's mask from shared memory (128 bytes in the
+        // 128-byte swizzle: piece c at c ^ (row & 7)); rows past Tq and keys
+        // past Tkv were filled with zeros (those keys are set to -inf below)
+        const int ms = 2 * t + (jj & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(&m_full[ms], (jj >> 1) & 1, abort_v, args.err));
+        if (!ok) break;
+        const uint8_t* mrow_s = sMask + ms * L::kMaskBytes + (row & (kRowsPerTile - 1)) * 128;
+        const uint64_t l2e = f2(kLog2e, kLog2e);
+#pragma unroll
+        for (int c = 0; c < BN; c += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(mrow_s + (((c >> 3) ^ (row & 7)) << 4));
+          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)  // bf16 pair -> fp32 pair by moving each half to the top 16 bits
+            x2[c / 2 + u] = f2_fma(f2u(wv[u] << 16, wv[u] & 0xFFFF0000u), l2e, x2[c / 2 + u]);
+        }
+        mbar_arrive(&m_empty[ms]);
       } else if constexpr (MASK == TC_BOOL) {
         if (row_valid) {
           const uint8_t* mp = static_cast<const uint8_t*>(args.mask) + mrow + j0;
@@ -876,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 // ---------------------------------------------------------------- host side
 template <int D, int BN, int KW, int MASK, int NS>
 cudaError_t launch_one(const TcArgs& a, dim3 grid, cudaStream_t stream) {
-  using L = Layout<D, BN, KW, NS>;
+  using L = Layout<D, BN, KW, NS, MASK == TC_FLOAT_TMA>;
   auto kern = flash_fwd_tc<D, BN, KW, MASK, NS>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -1051,7 +1105,20 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   dim3 grid((unsigned)(a.n_full + n_split_units * a.n_split), 1u, 1u);
   if (!p.use_rel) {
     if (p.d == 64) return dispatch_mask<64, 128, 0, 3>(mk, a, grid, stream);
-    if (BN_of(p) == 64) return dispatch_mask<128, 64, 0, 4>(mk, a, grid, stream);
+    if (BN_of(p) == 64) {
+      // an additive mask whose rows TMA can read: mask tiles staged by TMA
+      // (three K/V stages leave room for two mask stages per query tile)
+      if (mk == TC_FLOAT && a.mask_vec) {
+        const uint64_t hm = p.msh ? (uint64_t)p.Hq : 1, bm = p.msb ? (uint64_t)p.B : 1;
+        const uint64_t sq = 2 * (uint64_t)p.msq;
+        const uint64_t sh = p.msh ? 2 * (uint64_t)p.msh : sq * (uint64_t)p.Tq;
+        const uint64_t sb = p.msb ? 2 * (uint64_t)p.msb : sh * hm;
+        if (make_tmap_4d(&a.tm, p.mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.Tkv, p.Tq, hm, bm, sq, sh, sb, 64,
+                         kRowsPerTile, true))
+          return launch_one<128, 64, 0, TC_FLOAT_TMA, 3>(a, grid, stream);
+      }
+      return dispatch_mask<128, 64, 0, 4>(mk, a, grid, stream);
+    }
     return dispatch_mask<128, 128, 0, 2>(mk, a, grid, stream);
   }
   switch (p.kw_n) {
