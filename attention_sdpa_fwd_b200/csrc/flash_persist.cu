@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
       if (!ok) break;
       tc_fence_after();
       uint8_t* stage = sQ + (it & 1) * L::kQBuf + t * L::kQBytes + (warp & 3) * 32 * 128;
-      tile::stage_o_row_sw128<kD>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, stage + lane * 128, lane);
+      tile::stage_o_row_sw128<kD>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, stage + lane * 128, lane, 0);
       fence_proxy_async_shared();
       __syncwarp();
       if (lane == 0) {

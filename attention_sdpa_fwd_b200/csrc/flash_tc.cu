@@ -69,6 +69,7 @@ enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3, TC_FLOAT_TMA
 struct TcArgs {
   CUtensorMap tq, tk, tv, trh, trw;
   CUtensorMap tm;  // TC_FLOAT_TMA: the mask as (key, query row, head, batch), 64 x 128 boxes
+  CUtensorMap to;  // out, 64-column x 32-row boxes: a softmax warp stores its rows by TMA
   void* out;
   long long sob, soh, sot;  // element strides of out (batch, head, token)
   float* lse;
@@ -807,7 +808,24 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           if (args.lse) args.lse[zq * args.Tq + qi] = -INFINITY;
         }
       } else if (ok) {
-        tile::store_o_row<D>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, orow, row_valid);
+        // O / l as bf16 rows staged in this query tile's Q buffer (dead: the
+        // tile's last Q.K^T has completed), in the Q load's own 128-byte
+        // swizzle, then one TMA store per 64-column panel of the warp's 32
+        // rows (rows past Tq are not written)
+        uint8_t* stage = sQ + t * L::kQBytes + (warp & 3) * 32 * 128;
+        tile::stage_o_row_sw128<D>(o_addr, l_run > 0.f ? 1.f / l_run : 0.f, stage + lane * 128, lane,
+                                   kRowsPerTile * 128);
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          const int r0 = q0 + t * kRowsPerTile + (warp & 3) * 32;
+          if (r0 < args.Tq) {
+            for (int pnl = 0; pnl < L::kPanels; ++pnl)
+              tma_store_4d(&args.to, stage + pnl * kRowsPerTile * 128, pnl * 64, r0, h, b);
+            bulk_commit();
+            bulk_wait_read_all();  // shared memory must stay until the stores have read it
+          }
+        }
         if (row_valid && args.lse)
           args.lse[zq * args.Tq + qi] = l_run > 0.f ? m_run * kLn2 + logf(l_run) : -INFINITY;
       }
@@ -992,7 +1010,7 @@ int tc_check(const Params& p, sdpa_dtype_t dtype) {
   // TMA: byte strides multiples of 16 and below 2^40
   if (!strides_multiple_of(p, 8)) return SDPA_ERR_MISALIGNED;
   {
-    const long long s[9] = {p.sqb, p.sqh, p.sqt, p.skb, p.skh, p.skt, p.svb, p.svh, p.svt};
+    const long long s[12] = {p.sqb, p.sqh, p.sqt, p.skb, p.skh, p.skt, p.svb, p.svh, p.svt, p.sob, p.soh, p.sot};
     for (long long x : s)
       if (x >= (1LL << 38)) return SDPA_ERR_UNSUPPORTED;
   }
@@ -1067,6 +1085,7 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
     ok = ok && make_tmap_3d(&a.trh, p.rel_h, bf, 2, p.d, nh, 1, rowb, rowb * nh, 64, a.rel_n, true);
     ok = ok && make_tmap_3d(&a.trw, p.rel_w, bf, 2, p.d, nw, 1, rowb, rowb * nw, 64, a.rel_n, true);
   }
+  ok = ok && make_tmap_4d(&a.to, p.out, bf, p.d, p.Tq, p.Hq, p.B, 2 * p.sot, 2 * p.soh, 2 * p.sob, 64, 32, true);
   if (!ok) return cudaErrorInvalidValue;
   a.out = p.out;
   a.sob = p.sob; a.soh = p.soh; a.sot = p.sot;

@@ -107,13 +107,15 @@ __device__ __forceinline__ void store_o_row(uint32_t o_addr, float inv, __nv_bfl
   }
 }
 
-// The same epilogue into shared memory for a TMA store: the row's 64 bf16
-// values (128 bytes) at srow in the 128-byte swizzle of a tensor map with
-// 128-byte rows -- 16-byte piece c at position c ^ (r & 7), r the row's index
-// in its 1024-byte-aligned block (so a warp's 32 rows hit every bank group).
+// The same epilogue into shared memory for a TMA store: the row's D bf16
+// values as 128-byte pieces of 64 columns (panel p at srow + p * panel_bytes),
+// each in the 128-byte swizzle of a tensor map with 128-byte rows -- 16-byte
+// chunk c at position c ^ (r & 7), r the row's index in its 1024-byte-aligned
+// block (so a warp's 32 rows hit every bank group).
 template <int D>
-__device__ __forceinline__ void stage_o_row_sw128(uint32_t o_addr, float inv, uint8_t* srow, int r) {
-  static_assert(D == 64, "one 128-byte row");
+__device__ __forceinline__ void stage_o_row_sw128(uint32_t o_addr, float inv, uint8_t* srow, int r,
+                                                  int panel_bytes) {
+  static_assert(D % 64 == 0, "whole 64-column panels");
 #pragma unroll
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t v[32];
@@ -126,8 +128,9 @@ __device__ __forceinline__ void stage_o_row_sw128(uint32_t o_addr, float inv, ui
       w.y = pack_bf16x2(__uint_as_float(v[c + 2]) * inv, __uint_as_float(v[c + 3]) * inv);
       w.z = pack_bf16x2(__uint_as_float(v[c + 4]) * inv, __uint_as_float(v[c + 5]) * inv);
       w.w = pack_bf16x2(__uint_as_float(v[c + 6]) * inv, __uint_as_float(v[c + 7]) * inv);
-      const int piece = (c0 + c) >> 3;
-      *reinterpret_cast<uint4*>(srow + ((piece ^ (r & 7)) << 4)) = w;
+      const int col = c0 + c;  // first of the 8 columns
+      const int chunk = (col & 63) >> 3;
+      *reinterpret_cast<uint4*>(srow + (col >> 6) * panel_bytes + ((chunk ^ (r & 7)) << 4)) = w;
     }
   }
 }
