@@ -61,14 +61,14 @@ constexpr int kRelHMax = 64;  // key-grid height limit of the tensor-core rel-po
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// TC_FLOAT_TMA: the additive bf16 mask of TC_FLOAT, 64-key tiles brought into
-// shared memory by the producer warp (TMA, two stages per query tile) instead
-// of per-row global loads in the softmax warps.
-enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3, TC_FLOAT_TMA = 4 };
+// TC_FLOAT_TMA / TC_BOOL_TMA: the mask tensors of TC_FLOAT / TC_BOOL, 64-key
+// tiles brought into shared memory by the producer warp (TMA, two stages per
+// query tile) instead of per-row global loads in the softmax warps.
+enum TcMask { TC_NONE = 0, TC_RANGE = 1, TC_FLOAT = 2, TC_BOOL = 3, TC_FLOAT_TMA = 4, TC_BOOL_TMA = 5 };
 
 struct TcArgs {
   CUtensorMap tq, tk, tv, trh, trw;
-  CUtensorMap tm;  // TC_FLOAT_TMA: the mask as (key, query row, head, batch), 64 x 128 boxes
+  CUtensorMap tm;  // TC_*_TMA: the mask as (key, query row, head, batch), 64 x 128 boxes
   CUtensorMap to;  // out, 64-column x 32-row boxes: a softmax warp stores its rows by TMA
   void* out;
   long long sob, soh, sot;  // element strides of out (batch, head, token)
@@ -97,7 +97,7 @@ struct TcArgs {
   int* err;
 };
 
-template <int D, int BN, int KW, int NS, bool MT = false>
+template <int D, int BN, int KW, int NS, int MT = 0>  // MT: bytes per mask element (0: no mask tiles)
 struct Layout {
   static constexpr int kPanels = D / 64;
   static constexpr int kQBytes = kPanels * kRowsPerTile * 128;  // one Q tile
@@ -107,7 +107,7 @@ struct Layout {
   static constexpr int oK = oQ + 2 * kQBytes;
   static constexpr int oV = oK + NS * kKVBytes;
   static constexpr int oRel = oV + NS * kKVBytes;
-  static constexpr int kMaskBytes = MT ? kRowsPerTile * BN * 2 : 0;  // one query tile's mask tile (bf16)
+  static constexpr int kMaskBytes = kRowsPerTile * BN * MT;  // one query tile's mask tile
   static constexpr int oMask = oRel + kRelRows * 256 * 4;            // [query tile][stage]
   static constexpr int oBar = oMask + 4 * kMaskBytes;
   static constexpr int kBars = 4 * NS + 20 + (MT ? 8 : 0);
@@ -123,9 +123,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 
 template <int D, int BN, int KW, int MASK, int NS>
 __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constant__ TcArgs args) {
-  constexpr bool kMaskTma = (MASK == TC_FLOAT_TMA);
-  static_assert(!kMaskTma || (BN == 64 && KW == 0), "TMA mask tiles: 64 keys of 128-byte rows");
-  using L = Layout<D, BN, KW, NS, kMaskTma>;
+  constexpr bool kMaskTma = (MASK == TC_FLOAT_TMA || MASK == TC_BOOL_TMA);
+  constexpr int kMaskElem = MASK == TC_FLOAT_TMA ? 2 : (MASK == TC_BOOL_TMA ? 1 : 0);
+  static_assert(!kMaskTma || (BN == 64 && KW == 0), "TMA mask tiles: 64 keys per row");
+  using L = Layout<D, BN, KW, NS, kMaskElem>;
   // head_dim 64 leaves 128 TMEM columns free: P_A [384,448), P_B [448,512) get
   // their own columns, so S_t(j+1) = Q_t.K_{j+1}^T can be issued as soon as
   // softmax t has read S_t(j), before P_t(j) exists.  At head_dim 128, P_t
@@ -701,21 +702,36 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           }
         }
       } else if constexpr (kMaskTma) {
-        // this row of the tile's mask from shared memory (128 bytes in the
-        // 128-byte swizzle: piece c at c ^ (row & 7)); rows past Tq and keys
-        // past Tkv were filled with zeros (those keys are set to -inf below)
+        // this row of the tile's mask from shared memory: 128 bytes of bf16 in
+        // the 128-byte swizzle (16-byte piece c at c ^ (row & 7)), or 64 bytes
+        // of bool in the 64-byte swizzle (piece c at c ^ ((row >> 1) & 3)).
+        // Rows past Tq and keys past Tkv were filled with zeros: a zero bool
+        // hides a key, which is right for those keys (and their rows are
+        // never stored); float keys past Tkv are set to -inf below.
         const int ms = 2 * t + (jj & 1);
         ok = __all_sync(0xffffffffu, mbar_wait(&m_full[ms], (jj >> 1) & 1, abort_v, args.err));
         if (!ok) break;
-        const uint8_t* mrow_s = sMask + ms * L::kMaskBytes + (row & (kRowsPerTile - 1)) * 128;
-        const uint64_t l2e = f2(kLog2e, kLog2e);
+        const int rt = row & (kRowsPerTile - 1);
+        const uint8_t* mrow_s = sMask + ms * L::kMaskBytes + rt * (BN * kMaskElem);
+        if constexpr (MASK == TC_FLOAT_TMA) {
+          const uint64_t l2e = f2(kLog2e, kLog2e);
 #pragma unroll
-        for (int c = 0; c < BN; c += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(mrow_s + (((c >> 3) ^ (row & 7)) << 4));
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+          for (int c = 0; c < BN; c += 8) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(mrow_s + (((c >> 3) ^ (rt & 7)) << 4));
+            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u)  // bf16 pair -> fp32 pair by moving each half to the top 16 bits
-            x2[c / 2 + u] = f2_fma(f2u(wv[u] << 16, wv[u] & 0xFFFF0000u), l2e, x2[c / 2 + u]);
+            for (int u = 0; u < 4; ++u)  // bf16 pair -> fp32 pair by moving each half to the top 16 bits
+              x2[c / 2 + u] = f2_fma(f2u(wv[u] << 16, wv[u] & 0xFFFF0000u), l2e, x2[c / 2 + u]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; c += 16) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(mrow_s + (((c >> 4) ^ ((rt >> 1) & 3)) << 4));
+            const uint8_t* e = reinterpret_cast<const uint8_t*>(&raw);
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              if (e[u] == 0) set_ninf(c + u);
+          }
         }
         mbar_arrive(&m_empty[ms]);
       } else if constexpr (MASK == TC_BOOL) {
@@ -948,7 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
 // ---------------------------------------------------------------- host side
 template <int D, int BN, int KW, int MASK, int NS>
 cudaError_t launch_one(const TcArgs& a, dim3 grid, cudaStream_t stream) {
-  using L = Layout<D, BN, KW, NS, MASK == TC_FLOAT_TMA>;
+  using L = Layout<D, BN, KW, NS, MASK == TC_FLOAT_TMA ? 2 : (MASK == TC_BOOL_TMA ? 1 : 0)>;
   auto kern = flash_fwd_tc<D, BN, KW, MASK, NS>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -1125,16 +1141,20 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   if (!p.use_rel) {
     if (p.d == 64) return dispatch_mask<64, 128, 0, 3>(mk, a, grid, stream);
     if (BN_of(p) == 64) {
-      // an additive mask whose rows TMA can read: mask tiles staged by TMA
+      // a mask tensor whose rows TMA can read: mask tiles staged by TMA
       // (three K/V stages leave room for two mask stages per query tile)
-      if (mk == TC_FLOAT && a.mask_vec) {
+      if ((mk == TC_FLOAT || mk == TC_BOOL) && a.mask_vec) {
+        const uint64_t es = mk == TC_FLOAT ? 2 : 1;
         const uint64_t hm = p.msh ? (uint64_t)p.Hq : 1, bm = p.msb ? (uint64_t)p.B : 1;
-        const uint64_t sq = 2 * (uint64_t)p.msq;
-        const uint64_t sh = p.msh ? 2 * (uint64_t)p.msh : sq * (uint64_t)p.Tq;
-        const uint64_t sb = p.msb ? 2 * (uint64_t)p.msb : sh * hm;
-        if (make_tmap_4d(&a.tm, p.mask, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.Tkv, p.Tq, hm, bm, sq, sh, sb, 64,
-                         kRowsPerTile, true))
-          return launch_one<128, 64, 0, TC_FLOAT_TMA, 3>(a, grid, stream);
+        const uint64_t sq = es * (uint64_t)p.msq;
+        const uint64_t sh = p.msh ? es * (uint64_t)p.msh : sq * (uint64_t)p.Tq;
+        const uint64_t sb = p.msb ? es * (uint64_t)p.msb : sh * hm;
+        const bool fl = mk == TC_FLOAT;
+        if (make_tmap_4d(&a.tm, p.mask, fl ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, p.Tkv,
+                         p.Tq, hm, bm, sq, sh, sb, 64, kRowsPerTile,
+                         fl ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+          return fl ? launch_one<128, 64, 0, TC_FLOAT_TMA, 3>(a, grid, stream)
+                    : launch_one<128, 64, 0, TC_BOOL_TMA, 3>(a, grid, stream);
       }
       return dispatch_mask<128, 64, 0, 4>(mk, a, grid, stream);
     }

@@ -30,7 +30,7 @@ inline EncodeTiledFn encode_tiled_fn() {
 }
 
 // Encoded maps, cached by every argument of the encode call (base address,
-// type, rank, extents, byte strides, box, swizzle).  A map is a pure function
+// type, rank, extents, byte strides, box, swizzle mode).  A map is a pure function
 // of those arguments, so a repeated call on the same tensor -- the usual case
 // for a layer run step after step -- copies the cached 128-byte map instead of
 // calling the driver.  Fixed size, round-robin replacement, one mutex.
@@ -75,7 +75,7 @@ inline TmapCache& tmap_cache() {
 }
 
 inline TmapKey tmap_key(const void* base, CUtensorMapDataType dt, int rank, const cuuint64_t* dims,
-                        const cuuint64_t* strides, const cuuint32_t* box, bool swizzle128) {
+                        const cuuint64_t* strides, const cuuint32_t* box, int swizzle) {
   TmapKey k;
   memset(&k, 0, sizeof(k));  // padding included: keys compare with memcmp
   k.base = base;
@@ -85,22 +85,22 @@ inline TmapKey tmap_key(const void* base, CUtensorMapDataType dt, int rank, cons
   k.box[1] = box[1];
   k.dt = (int)dt;
   k.rank = rank;
-  k.swizzle = swizzle128 ? 1 : 0;
+  k.swizzle = swizzle;
   return k;
 }
 
 // One encode through the cache; false if the driver rejects the map.
 inline bool encode_cached(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int rank,
                           const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
-                          bool swizzle128) {
-  const TmapKey key = tmap_key(base, dt, rank, dims, strides, box, swizzle128);
+                          CUtensorMapSwizzle swz) {
+  const TmapKey key = tmap_key(base, dt, rank, dims, strides, box, (int)swz);
   if (tmap_cache().find(key, map)) return true;
   EncodeTiledFn fn = encode_tiled_fn();
   if (fn == nullptr) return false;
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
   tmap_cache().put(key, *map);
   return true;
@@ -118,21 +118,29 @@ inline bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType
   cuuint64_t strides[2] = {s1, s2};
   cuuint32_t box[3] = {b0, b1, 1};
   (void)elem_bytes;
-  return encode_cached(map, base, dt, 3, dims, strides, box, swizzle128);
+  return encode_cached(map, base, dt, 3, dims, strides, box,
+                       swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // 4-D map over a tensor of `elem_bytes` elements with dims {n0, n1, n2, n3}
 // (dim0 contiguous) and byte strides s1, s2, s3 of dims 1..3, in any order of
 // magnitude (e.g. head_dim, token, head, batch of a "bshd" tensor); box
-// {b0, b1, 1, 1}; 128-byte swizzle when asked.  Out-of-range elements of a box
-// read as zero.  Returns false if the driver rejects the map.
+// {b0, b1, 1, 1}; the given swizzle mode (or, with a bool, the 128-byte
+// swizzle when asked).  Out-of-range elements of a box read as zero.  Returns
+// false if the driver rejects the map.
 inline bool make_tmap_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t n0,
                          uint64_t n1, uint64_t n2, uint64_t n3, uint64_t s1, uint64_t s2, uint64_t s3,
-                         uint32_t b0, uint32_t b1, bool swizzle128) {
+                         uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
   cuuint64_t dims[4] = {n0, n1, n2, n3};
   cuuint64_t strides[3] = {s1, s2, s3};
   cuuint32_t box[4] = {b0, b1, 1, 1};
-  return encode_cached(map, base, dt, 4, dims, strides, box, swizzle128);
+  return encode_cached(map, base, dt, 4, dims, strides, box, swz);
+}
+inline bool make_tmap_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t n0,
+                         uint64_t n1, uint64_t n2, uint64_t n3, uint64_t s1, uint64_t s2, uint64_t s3,
+                         uint32_t b0, uint32_t b1, bool swizzle128) {
+  return make_tmap_4d(map, base, dt, n0, n1, n2, n3, s1, s2, s3, b0, b1,
+                      swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace sdpa

@@ -97,6 +97,22 @@ CASES = [
        mask_neg_inf_frac=0.2, mask_heads=1, seed=36),
     S_("float_bf16_d128_odd_tiles", BF16, 2, 3, 3, 200, 300, 128, mask_kind=W.MASK_FLOAT, mask_std=2.0,
        mask_neg_inf_frac=0.1, mask_heads=3, seed=37),
+    # key counts that are multiples of 8 (16-byte mask rows): the mask tiles
+    # reach shared memory by TMA -- broadcast over heads with a ragged last
+    # key tile and query block, one mask per head, a single partial tile
+    S_("float_bf16_d128_tma_bcast", BF16, 2, 4, 2, 260, 296, 128, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=1, seed=38),
+    S_("float_bf16_d128_tma_perhead", BF16, 1, 3, 1, 130, 200, 128, mask_kind=W.MASK_FLOAT, mask_std=2.0,
+       mask_neg_inf_frac=0.3, mask_heads=3, seed=39),
+    S_("float_bf16_d128_tma_one_tile", BF16, 1, 2, 2, 40, 40, 128, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=2, seed=49),
+    # boolean masks with 16-byte rows (key counts that are multiples of 16):
+    # the same TMA tiles, in the 64-byte swizzle; one mask per head with a
+    # ragged last tile, and a mostly hidden one with fully masked rows
+    S_("bool_bf16_d128_tma_perhead", BF16, 1, 2, 1, 150, 208, 128, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.6,
+       mask_heads=2, seed=56),
+    S_("bool_bf16_d128_tma_sparse", BF16, 2, 2, 2, 70, 48, 128, mask_kind=W.MASK_BOOL, mask_neg_inf_frac=0.9,
+       mask_heads=1, seed=57),
     # more query blocks than SMs: the persistent form walks several per CTA
     # (consecutive units of one CTA differ in window, head and query block)
     S_("persist_relpos_14x14_many", BF16, 40, 4, 4, 196, 196, 64, q_hw=(14, 14), k_hw=(14, 14), rel_std=0.5,
