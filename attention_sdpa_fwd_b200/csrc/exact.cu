@@ -120,14 +120,24 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     l = l * corr + psum;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] *= corr;
+    // the value sum over the chunk's keys, eight at a time: the eight V loads
+    // go out together, then the eight FMAs (one round trip per eight keys)
     const int nk = (int)((hi - j0) < 32 ? (hi - j0) : 32);
-    for (int t = 0; t < nk; ++t) {
-      const float pt = __shfl_sync(0xffffffffu, pj, t);
-      if (owns_cols && dcheck_kv(p, b, hk, j0 + t)) {
-        const T* vr = vb + (j0 + t) * p.svt + col0;
+    for (int t0 = 0; t0 < nk; t0 += 8) {
+      float pt[8], vv[8][CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[c] = fmaf(pt, to_f32(vr[c]), acc[c]);
+      for (int u = 0; u < 8; ++u) {
+        const int t = t0 + u;  // < 32
+        pt[u] = __shfl_sync(0xffffffffu, pj, t);
+        const bool live = t < nk && owns_cols && dcheck_kv(p, b, hk, j0 + t);
+        const T* vr = vb + (j0 + (live ? t : 0)) * p.svt + col0;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) vv[u][c] = live ? to_f32(vr[c]) : 0.f;
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[c] = fmaf(pt[u], vv[u][c], acc[c]);
     }
     m = mnew;
   }
