@@ -201,6 +201,171 @@ __global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p, int h
   if (p.lse) p.lse[zq * p.Tq + i] = l > 0.f ? m * kLn2 + logf(l) : -INFINITY;
 }
 
+// ------------------------------------------------------------------ tensor-core fragments
+// mma.sync m16n8k16, bf16 operands, fp32 accumulate.  Thread (g, t) =
+// (lane / 4, lane % 4) of a warp holds: of a 16x16 A tile, rows g and g + 8 at
+// columns 2t, 2t + 1 (registers 0, 1) and 2t + 8, 2t + 9 (registers 2, 3); of
+// a 16x8 B tile, column g at rows 2t, 2t + 1 (register 0) and 2t + 8, 2t + 9
+// (register 1); of the 16x8 fp32 accumulator, rows g (c0, c1) and g + 8
+// (c2, c3) at columns 2t, 2t + 1.  The S = Q K^T accumulators of two 8-key
+// tiles, packed to bf16, are exactly the A operand of O += P V over those 16
+// keys, so P never leaves registers.  Operands come from shared memory
+// through ldmatrix.
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+               "{%8, %9}, {%0, %1, %2, %3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Byte offset of 16-byte half h (d 0..7 or 8..15) of row r in a [rows][16]
+// bf16 array: halves swap every 4 rows, so the 8 rows one ldmatrix matrix
+// reads hit all 32 banks once.
+__device__ __forceinline__ uint32_t sw32(int r, int h) { return (uint32_t)(r * 32 + ((h ^ ((r >> 2) & 1)) << 4)); }
+
+// The A operand (rows row0 .. row0 + 15) of a [rows][16] bf16 array at base.
+__device__ __forceinline__ void ldsm_a(uint32_t (&a)[4], uint32_t base, int row0, int lane) {
+  ldsm_x4(a, base + sw32(row0 + (lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4));
+}
+// K of keys key0 .. key0 + 15 as the B operands of two 8-key tiles of S = Q K^T:
+// r[0], r[1] for keys key0 .. + 7, r[2], r[3] for keys key0 + 8 .. + 15.
+__device__ __forceinline__ void ldsm_k(uint32_t (&r)[4], uint32_t base, int key0, int lane) {
+  ldsm_x4(r, base + sw32(key0 + (lane & 7) + (lane >> 4) * 8, (lane >> 3) & 1));
+}
+// V of keys key0 .. key0 + 15 as the B operands of O += P V: r[0], r[1] for
+// value columns 0 .. 7, r[2], r[3] for columns 8 .. 15.
+__device__ __forceinline__ void ldsm_v(uint32_t (&r)[4], uint32_t base, int key0, int lane) {
+  ldsm_x4_t(r, base + sw32(key0 + (lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4));
+}
+
+constexpr int kPartStride = 20;  // floats per row partial: 16 O, m, l, pad
+
+// One warp's partial of 16 query rows over NT tiles of 16 keys of a staged
+// part: S = Q K^T on the tensor cores from the staged bf16 rows (Q rows
+// qrow0 .. qrow0 + 15 of q_s; keys key0 .. key0 + 16 NT - 1 of k_s / v_s, of
+// which those at or past n are absent), the scores in log2 units with the
+// mask (the rows are query rows row0 .. row0 + 15, staged key kk is key
+// jg0 + kk of the problem), the softmax over the warp's keys, and O = P V with
+// P packed straight from the S accumulators.  For every row row0 + i < Tq,
+// writes the unnormalised O (16 values), the max m (log2 units) and the sum l
+// to wp + i * kPartStride.
+template <int NT>
+__device__ __forceinline__ void warp_slice_partial(const Params& p, int b, int h, uint32_t q_s, int qrow0,
+                                                   uint32_t k_s, uint32_t v_s, int key0, int n, long long jg0,
+                                                   long long row0, float* wp, int lane, float sl) {
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t qa[4];
+  ldsm_a(qa, q_s, qrow0, lane);
+  float x[NT][2][4];
+#pragma unroll
+  for (int c = 0; c < NT; ++c) {
+    uint32_t kf[4];
+    ldsm_k(kf, k_s, key0 + 16 * c, lane);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      x[c][u][0] = x[c][u][1] = x[c][u][2] = x[c][u][3] = 0.f;
+      mma16816(x[c][u], qa, kf[2 * u], kf[2 * u + 1]);
+    }
+  }
+  // scores in log2 units with the mask; absent keys and rows past Tq score -inf
+  const long long mrow_base = (long long)b * p.msb + (long long)h * p.msh;
+#pragma unroll
+  for (int c = 0; c < NT; ++c)
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const long long row = row0 + g + (e >> 1) * 8;
+        const int kk = key0 + 16 * c + 8 * u + 2 * t + (e & 1);
+        float v = x[c][u][e] * sl;
+        if (kk >= n || row >= p.Tq)
+          v = -INFINITY;
+        else
+          v += mask_term(p, mrow_base + row * p.msq, row, jg0 + kk);
+        x[c][u][e] = v;
+      }
+  float mr[2], lr[2] = {0.f, 0.f}, o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < NT; ++c)
+      mx = fmaxf(mx, fmaxf(fmaxf(x[c][0][2 * r], x[c][0][2 * r + 1]), fmaxf(x[c][1][2 * r], x[c][1][2 * r + 1])));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mr[r] = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  }
+#pragma unroll
+  for (int c = 0; c < NT; ++c) {
+    uint32_t pa[4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float mu = mr[r] == -INFINITY ? 0.f : mr[r];  // nothing visible: every p is 0
+      const float p00 = sm100::ex2_approx(x[c][0][2 * r] - mu), p01 = sm100::ex2_approx(x[c][0][2 * r + 1] - mu);
+      const float p10 = sm100::ex2_approx(x[c][1][2 * r] - mu), p11 = sm100::ex2_approx(x[c][1][2 * r + 1] - mu);
+      lr[r] += (p00 + p01) + (p10 + p11);
+      pa[r] = pack2(p00, p01);      // keys 2t, 2t + 1 of the 16
+      pa[r + 2] = pack2(p10, p11);  // keys 8 + 2t, 9 + 2t
+    }
+    uint32_t vf[4];
+    ldsm_v(vf, v_s, key0 + 16 * c, lane);
+    mma16816(o[0], pa, vf[0], vf[1]);
+    mma16816(o[1], pa, vf[2], vf[3]);
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int i = g + 8 * r;
+    float L = lr[r];
+    L += __shfl_xor_sync(0xffffffffu, L, 1);
+    L += __shfl_xor_sync(0xffffffffu, L, 2);
+    if (row0 + i >= p.Tq) continue;
+    float* pr = wp + i * kPartStride;
+    pr[2 * t] = o[0][2 * r];
+    pr[2 * t + 1] = o[0][2 * r + 1];
+    pr[8 + 2 * t] = o[1][2 * r];
+    pr[9 + 2 * t] = o[1][2 * r + 1];
+    if (t == 0) {
+      pr[16] = mr[r];
+      pr[17] = L;
+    }
+  }
+}
+
+// The CTA's partial of a row from its warps' partials ws[k * wstride] (k <
+// 8, each O, m, l as warp_slice_partial writes them): warp-collective; lane
+// c < 16 returns column c of O relative to the returned max M, with den the
+// matching sum.
+__device__ __forceinline__ void combine_warp_partials(const float* ws, int wstride, int lane, float& num,
+                                                      float& M, float& den) {
+  float Mk = -INFINITY, lk = 0.f;
+  if (lane < 8) {
+    Mk = ws[lane * wstride + 16];
+    lk = ws[lane * wstride + 17];
+  }
+  M = lk > 0.f ? Mk : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float wk = lk > 0.f ? sm100::ex2_approx(Mk - M) : 0.f;
+  den = wk * lk;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  num = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float w_k = __shfl_sync(0xffffffffu, wk, k);
+    if (lane < D16 && w_k > 0.f) num = fmaf(w_k, ws[k * wstride + lane], num);
+  }
+}
+
 // ------------------------------------------------------------------ split_kv
 constexpr int kSplitThreads = 256;  // 8 warps: one query row per warp at a time
 constexpr int kSplitChunk = 256;    // keys per CTA part (at most)
@@ -214,123 +379,70 @@ struct SplitArgs {
   int* ws_cnt;     // [B*Hq] tickets, zero between launches
 };
 
-__global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a) {
+constexpr int kWsRows = 32;  // query rows per block of the workspace kernel (two 16-row tiles)
+
+__global__ void __launch_bounds__(kSplitThreads, 3) split_kv_kernel(SplitArgs a) {
   const Params& p = a.p;
-  // key t's row as four float4 at [t][f ^ ((t >> 1) & 3)]: eight consecutive
-  // lanes reading the same f of consecutive keys hit all 32 banks once
-  __shared__ float4 sk[kSplitChunk][D16 / 4];
-  __shared__ float4 sv[kSplitChunk][D16 / 4];
+  constexpr int kWarps = kSplitThreads / 32;
+  static_assert(kSplitChunk == kSplitThreads && kSplitChunk == kWarps * 32, "a key per thread, 32 per warp");
+  __shared__ __align__(128) uint8_t sk[kSplitChunk * 32];  // staged K rows (bf16, swizzled halves)
+  __shared__ __align__(128) uint8_t sv[kSplitChunk * 32];
+  __shared__ __align__(128) uint8_t sq[kWsRows * 32];
+  __shared__ float warp_s[kWarps][kWsRows][kPartStride];
   __shared__ int s_last;
   const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.group;
   const long long zq = (long long)b * p.Hq + h;
   const long long j0 = (long long)part * a.chunk;
   const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, 0);
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, 0);
-  for (int t = threadIdx.x; t < n; t += kSplitThreads) {
-    if (!dcheck_kv(p, b, hk, j0 + t)) continue;
-    float f[D16];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt)), f);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kb + (j0 + t) * p.skt) + 1), f + 8);
-#pragma unroll
-    for (int c = 0; c < D16; c += 4) sk[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt)), f);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(vb + (j0 + t) * p.svt) + 1), f + 8);
-#pragma unroll
-    for (int c = 0; c < D16; c += 4) sv[t][(c / 4) ^ ((t >> 1) & 3)] = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t k_s = sm100::smem_u32(sk), v_s = sm100::smem_u32(sv), q_s = sm100::smem_u32(sq);
+  {
+    // stage this part's K and V rows, one key per thread (zeros past the part)
+    uint4 k0 = make_uint4(0, 0, 0, 0), k1 = k0, v0 = k0, v1 = k0;
+    if (tid < n && dcheck_kv(p, b, hk, j0 + tid)) {
+      const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + k_off(p, b, hk, j0 + tid));
+      const uint4* vr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v) + v_off(p, b, hk, j0 + tid));
+      k0 = __ldg(kr);
+      k1 = __ldg(kr + 1);
+      v0 = __ldg(vr);
+      v1 = __ldg(vr + 1);
+    }
+    *reinterpret_cast<uint4*>(sk + sw32(tid, 0)) = k0;
+    *reinterpret_cast<uint4*>(sk + sw32(tid, 1)) = k1;
+    *reinterpret_cast<uint4*>(sv + sw32(tid, 0)) = v0;
+    *reinterpret_cast<uint4*>(sv + sw32(tid, 1)) = v1;
   }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl = p.scale * kLog2e;
-  for (int i = warp; i < p.Tq; i += kSplitThreads / 32) {
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, i);
-    float q[D16];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow)), q);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qrow) + 1), q + 8);
-    const long long mrow = (long long)b * p.msb + (long long)h * p.msh + (long long)i * p.msq;
-    float m = -INFINITY, l = 0.f, acc[D16];
-#pragma unroll
-    for (int c = 0; c < D16; ++c) acc[c] = 0.f;
-    // this lane's keys (lane, lane + 32, ... : at most kSplitChunk / 32 of
-    // them): scores, their max, then the sums
-    float sc[kSplitChunk / 32];
-#pragma unroll
-    for (int u = 0; u < kSplitChunk / 32; ++u) {
-      const int t = lane + 32 * u;
-      float x = -INFINITY;
-      if (t < n) {
-        x = 0.f;
-#pragma unroll
-        for (int c = 0; c < D16; c += 4) {
-          const float4 k4 = sk[t][(c / 4) ^ ((t >> 1) & 3)];
-          x = fmaf(q[c], k4.x, fmaf(q[c + 1], k4.y, fmaf(q[c + 2], k4.z, fmaf(q[c + 3], k4.w, x))));
-        }
-        x = x * sl + mask_term(p, mrow, i, j0 + t);
+  // query rows in blocks of 32: stage them, every warp's partial over its 32
+  // keys (tensor cores), then the CTA's partial of each row into the workspace
+  for (int rb = 0; rb < p.Tq; rb += kWsRows) {
+    if (tid < kWsRows) {
+      uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
+      if (rb + tid < p.Tq && dcheck_q(p, b, h, rb + tid)) {
+        const uint4* qr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + q_off(p, b, h, rb + tid));
+        q0 = __ldg(qr);
+        q1 = __ldg(qr + 1);
       }
-      sc[u] = x;
-      m = fmaxf(m, x);
+      *reinterpret_cast<uint4*>(sq + sw32(tid, 0)) = q0;
+      *reinterpret_cast<uint4*>(sq + sw32(tid, 1)) = q1;
     }
-    if (m != -INFINITY) {
+    __syncthreads();  // (the first block's barrier also covers the K/V staging)
 #pragma unroll
-      for (int u = 0; u < kSplitChunk / 32; ++u) {
-        const int t = lane + 32 * u;
-        const float pj = sm100::ex2_approx(sc[u] - m);  // 0 for -inf
-        l += pj;
-        if (t < n) {
-#pragma unroll
-          for (int c = 0; c < D16; c += 4) {
-            const float4 v4 = sv[t][(c / 4) ^ ((t >> 1) & 3)];
-            acc[c] = fmaf(pj, v4.x, acc[c]);
-            acc[c + 1] = fmaf(pj, v4.y, acc[c + 1]);
-            acc[c + 2] = fmaf(pj, v4.z, acc[c + 2]);
-            acc[c + 3] = fmaf(pj, v4.w, acc[c + 3]);
-          }
-        }
-      }
+    for (int m = 0; m < kWsRows / 16; ++m)
+      if (rb + 16 * m < p.Tq)
+        warp_slice_partial<2>(p, b, h, q_s, 16 * m, k_s, v_s, 32 * warp, n, j0, rb + 16 * m, &warp_s[warp][16 * m][0],
+                              lane, sl);
+    __syncthreads();
+    for (int i = warp; i < kWsRows && rb + i < p.Tq; i += kWarps) {
+      float num, M, den;
+      combine_warp_partials(&warp_s[0][i][0], kWsRows * kPartStride, lane, num, M, den);
+      const long long slot = (zq * a.nsplit + part) * p.Tq + rb + i;
+      if (!dcheck_idx(p.err, slot, (long long)p.B * p.Hq * a.nsplit * p.Tq)) continue;
+      if (lane < D16) __stcg(a.ws_o + slot * D16 + lane, num);
+      if (lane == 0) __stcg(a.ws_ml + slot, make_float2(M, den));
     }
-    // combine the 32 lanes
-    float M = m;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    l *= w;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    // sum the 16 columns over the 32 lanes as a butterfly reduce-scatter:
-    // at each step a lane keeps half of its columns and adds its partner's
-    // half (8 + 4 + 2 + 1 + 1 shuffles instead of 16 x 5); lane pair
-    // (2k, 2k+1) ends with column col = bits 4..1 of the lane
-#pragma unroll
-    for (int c = 0; c < D16; ++c) acc[c] *= w;
-    const long long slot = (zq * a.nsplit + part) * p.Tq + i;
-    const bool slot_ok = dcheck_idx(p.err, slot, (long long)p.B * p.Hq * a.nsplit * p.Tq);
-    float r8[8], r4[4], r2[2], r1;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const bool hi = lane & 16;
-      r8[k] = (hi ? acc[k + 8] : acc[k]) + __shfl_xor_sync(0xffffffffu, hi ? acc[k] : acc[k + 8], 16);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const bool hi = lane & 8;
-      r4[k] = (hi ? r8[k + 4] : r8[k]) + __shfl_xor_sync(0xffffffffu, hi ? r8[k] : r8[k + 4], 8);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const bool hi = lane & 4;
-      r2[k] = (hi ? r4[k + 2] : r4[k]) + __shfl_xor_sync(0xffffffffu, hi ? r4[k] : r4[k + 2], 4);
-    }
-    {
-      const bool hi = lane & 2;
-      r1 = (hi ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, hi ? r2[0] : r2[1], 2);
-    }
-    r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-    if ((lane & 1) == 0 && slot_ok) {
-      const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-      __stcg(a.ws_o + slot * D16 + col, r1);
-    }
-    if (lane == 0 && slot_ok) __stcg(a.ws_ml + slot, make_float2(M, l));
+    __syncthreads();  // the next block's staging overwrites sq and warp_s
   }
   // the last part of this (batch, head) to finish merges all parts.  The CTA
   // barrier orders every thread's stores before thread 0's gpu-scope fence
@@ -382,53 +494,6 @@ __global__ void __launch_bounds__(kSplitThreads, 4) split_kv_kernel(SplitArgs a)
   if (threadIdx.x == 0) a.ws_cnt[zq] = 0;  // ready for the next launch
 }
 
-// ------------------------------------------------------------------ tensor-core fragments
-// mma.sync m16n8k16, bf16 operands, fp32 accumulate.  Thread (g, t) =
-// (lane / 4, lane % 4) of a warp holds: of a 16x16 A tile, rows g and g + 8 at
-// columns 2t, 2t + 1 (registers 0, 1) and 2t + 8, 2t + 9 (registers 2, 3); of
-// a 16x8 B tile, column g at rows 2t, 2t + 1 (register 0) and 2t + 8, 2t + 9
-// (register 1); of the 16x8 fp32 accumulator, rows g (c0, c1) and g + 8
-// (c2, c3) at columns 2t, 2t + 1.  The S = Q K^T accumulators of two 8-key
-// tiles, packed to bf16, are exactly the A operand of O += P V over those 16
-// keys, so P never leaves registers.  Operands come from shared memory
-// through ldmatrix.
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-               "{%8, %9}, {%0, %1, %2, %3};"
-               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-// Byte offset of 16-byte half h (d 0..7 or 8..15) of row r in a [rows][16]
-// bf16 array: halves swap every 4 rows, so the 8 rows one ldmatrix matrix
-// reads hit all 32 banks once.
-__device__ __forceinline__ uint32_t sw32(int r, int h) { return (uint32_t)(r * 32 + ((h ^ ((r >> 2) & 1)) << 4)); }
-
-// The A operand (rows row0 .. row0 + 15) of a [rows][16] bf16 array at base.
-__device__ __forceinline__ void ldsm_a(uint32_t (&a)[4], uint32_t base, int row0, int lane) {
-  ldsm_x4(a, base + sw32(row0 + (lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4));
-}
-// K of keys key0 .. key0 + 15 as the B operands of two 8-key tiles of S = Q K^T:
-// r[0], r[1] for keys key0 .. + 7, r[2], r[3] for keys key0 + 8 .. + 15.
-__device__ __forceinline__ void ldsm_k(uint32_t (&r)[4], uint32_t base, int key0, int lane) {
-  ldsm_x4(r, base + sw32(key0 + (lane & 7) + (lane >> 4) * 8, (lane >> 3) & 1));
-}
-// V of keys key0 .. key0 + 15 as the B operands of O += P V: r[0], r[1] for
-// value columns 0 .. 7, r[2], r[3] for columns 8 .. 15.
-__device__ __forceinline__ void ldsm_v(uint32_t (&r)[4], uint32_t base, int key0, int lane) {
-  ldsm_x4_t(r, base + sw32(key0 + (lane & 7) + ((lane >> 3) & 1) * 8, lane >> 4));
-}
-
 // ------------------------------------------------------------------ split_kv over a cluster
 // The same split of the key axis, with the parts of one (batch, head) in one
 // thread-block cluster: each CTA leaves its partial (O, m, l) per query row
@@ -444,7 +509,6 @@ constexpr int kClusterMax = 8;      // portable cluster size
 constexpr int kClusterChunk = 512;  // keys per CTA (at most)
 constexpr int kWarpKeys = kClusterChunk / (kSplitThreads / 32);  // 64 keys per warp
 constexpr int kRowsMax = 64;        // query rows the partial areas hold
-constexpr int kPartStride = 20;     // floats per row partial: 16 O, m, l, pad
 // dynamic shared memory: K and V (bf16 rows), Q rows, the warps' partials,
 // the CTA's partials
 constexpr int kClK = 0, kClV = kClusterChunk * 32, kClQ = 2 * kClusterChunk * 32;
@@ -473,7 +537,7 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
   const long long zq = (long long)b * p.Hq + h;
   const long long j0 = (long long)part * a.chunk;
   const int n = (int)max(0LL, min((long long)a.chunk, (long long)p.Tkv - j0));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mrows = (p.Tq + 15) & ~15;  // query rows rounded up to whole 16-row tiles
   {
     // stage K and V rows tid and tid + 256 (zeros past the part) and Q rows
@@ -515,105 +579,14 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
   const float sl = p.scale * kLog2e;
   const int kw0 = warp * kWarpKeys;  // this warp's keys within the part: [kw0, kw0 + 64)
   float* wp = warp_s + warp * kRowsMax * kPartStride;
-  for (int row0 = 0; row0 < p.Tq; row0 += 16) {
-    uint32_t qa[4];
-    ldsm_a(qa, q_s, row0, lane);
-    float x[kWarpKeys / 16][2][4];
-#pragma unroll
-    for (int c = 0; c < kWarpKeys / 16; ++c) {
-      uint32_t kf[4];
-      ldsm_k(kf, k_s, kw0 + 16 * c, lane);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        x[c][u][0] = x[c][u][1] = x[c][u][2] = x[c][u][3] = 0.f;
-        mma16816(x[c][u], qa, kf[2 * u], kf[2 * u + 1]);
-      }
-    }
-    // scores in log2 units with the mask; keys past the part and rows past
-    // Tq score -inf
-    const long long mrow_base = (long long)b * p.msb + (long long)h * p.msh;
-#pragma unroll
-    for (int c = 0; c < kWarpKeys / 16; ++c)
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = row0 + g + (e >> 1) * 8;
-          const int kk = kw0 + 16 * c + 8 * u + 2 * t + (e & 1);
-          float v = x[c][u][e] * sl;
-          if (kk >= n || row >= p.Tq)
-            v = -INFINITY;
-          else
-            v += mask_term(p, mrow_base + (long long)row * p.msq, row, j0 + kk);
-          x[c][u][e] = v;
-        }
-    float mr[2], lr[2] = {0.f, 0.f}, o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kWarpKeys / 16; ++c)
-        mx = fmaxf(mx, fmaxf(fmaxf(x[c][0][2 * r], x[c][0][2 * r + 1]), fmaxf(x[c][1][2 * r], x[c][1][2 * r + 1])));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mr[r] = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    }
-#pragma unroll
-    for (int c = 0; c < kWarpKeys / 16; ++c) {
-      uint32_t pa[4];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float mu = mr[r] == -INFINITY ? 0.f : mr[r];  // nothing visible: every p is 0
-        const float p00 = sm100::ex2_approx(x[c][0][2 * r] - mu), p01 = sm100::ex2_approx(x[c][0][2 * r + 1] - mu);
-        const float p10 = sm100::ex2_approx(x[c][1][2 * r] - mu), p11 = sm100::ex2_approx(x[c][1][2 * r + 1] - mu);
-        lr[r] += (p00 + p01) + (p10 + p11);
-        pa[r] = pack2(p00, p01);      // keys 2t, 2t + 1 of the 16
-        pa[r + 2] = pack2(p10, p11);  // keys 8 + 2t, 9 + 2t
-      }
-      uint32_t vf[4];
-      ldsm_v(vf, v_s, kw0 + 16 * c, lane);
-      mma16816(o[0], pa, vf[0], vf[1]);
-      mma16816(o[1], pa, vf[2], vf[3]);
-    }
-    // this warp's partial of rows row0 + g and row0 + g + 8 (O unnormalised, m, l)
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = row0 + g + 8 * r;
-      float L = lr[r];
-      L += __shfl_xor_sync(0xffffffffu, L, 1);
-      L += __shfl_xor_sync(0xffffffffu, L, 2);
-      if (row >= p.Tq || !dcheck_idx(p.err, row, kRowsMax)) continue;
-      float* pr = wp + row * kPartStride;
-      pr[2 * t] = o[0][2 * r];
-      pr[2 * t + 1] = o[0][2 * r + 1];
-      pr[8 + 2 * t] = o[1][2 * r];
-      pr[9 + 2 * t] = o[1][2 * r + 1];
-      if (t == 0) {
-        pr[16] = mr[r];
-        pr[17] = L;
-      }
-    }
-  }
+  for (int row0 = 0; row0 < p.Tq; row0 += 16)
+    warp_slice_partial<kWarpKeys / 16>(p, b, h, q_s, row0, k_s, v_s, kw0, n, j0, row0, wp + row0 * kPartStride, lane,
+                                       sl);
   __syncthreads();
   // the CTA's partial of row i from its warps' (warp i % 8 combines row i)
   for (int i = warp; i < p.Tq; i += kWarps) {
-    float Mk = -INFINITY, lk = 0.f;
-    if (lane < kWarps) {
-      Mk = warp_s[(lane * kRowsMax + i) * kPartStride + 16];
-      lk = warp_s[(lane * kRowsMax + i) * kPartStride + 17];
-    }
-    float M = lk > 0.f ? Mk : -INFINITY;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float wk = lk > 0.f ? sm100::ex2_approx(Mk - M) : 0.f;
-    float den = wk * lk;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    float num = 0.f;
-#pragma unroll
-    for (int k = 0; k < kWarps; ++k) {
-      const float w_k = __shfl_sync(0xffffffffu, wk, k);
-      if (lane < D16 && w_k > 0.f) num = fmaf(w_k, warp_s[(k * kRowsMax + i) * kPartStride + lane], num);
-    }
+    float num, M, den;
+    combine_warp_partials(warp_s + i * kPartStride, kRowsMax * kPartStride, lane, num, M, den);
     if (lane < D16) part_s[i * kPartStride + lane] = num;
     if (lane == 0) {
       part_s[i * kPartStride + 16] = M;

@@ -25,6 +25,23 @@ EXPECTED = {
 }
 
 
+# head_dim-16 shapes on either side of the split-KV rule (Tkv >= 1024 and
+# Tq <= Tkv / 4), as (B, H, Tq, Tkv) -> family
+D16_RULE = [((4, 8, 8, 4096), "split_kv"), ((4, 8, 100, 8192), "split_kv"), ((4, 8, 256, 1024), "split_kv"),
+            ((4, 8, 257, 1024), "small_d"), ((4, 8, 8, 1023), "small_d"), ((4, 8, 4096, 8), "small_d"),
+            ((4, 8, 1024, 2048), "small_d")]
+
+
+@pytest.mark.parametrize("shape,family", D16_RULE)
+def test_auto_dispatch_head_dim_16(shape, family):
+    import bench
+    import torch
+    from attention_sdpa_fwd_b200 import workloads as W
+    B, H, Tq, Tkv = shape
+    sp = W.Spec("d16_rule", torch.bfloat16, B, H, H, Tq, Tkv, 16, 0.25, seed=0)
+    assert bench.auto_path_name(S, sp) == family
+
+
 @pytest.mark.parametrize("name", sorted(EXPECTED))
 def test_auto_dispatch_of_benchmark_workloads(name):
     import bench
