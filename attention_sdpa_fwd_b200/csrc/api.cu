@@ -183,12 +183,13 @@ int choose_path(const Problem& pr) {
     return SDPA_PATH_TCGEN05;
   }
   if (small_d_check(p, pr.dtype) == SDPA_OK) {
-    // a long key axis against at most a quarter as many query rows: split the
-    // keys over the SMs (tensor-core parts).  The small-d kernel costs a fixed
-    // time per 128-key round, so it keeps the short key axes and the long query
-    // axes (measured at 4 x 8 heads: 100 x 8192 rows x keys 97 against
-    // 1001 us, 512 x 4096 269 against 503 us, 512 x 1024 193 against 128 us).
-    if (p.Tkv >= 1024 && (long long)p.Tq * 4 <= p.Tkv) return SDPA_PATH_SPLIT_KV;
+    // a long key axis against at most a sixteenth as many query rows: split
+    // the keys over the SMs.  The small-d kernel walks the keys in rounds of
+    // 128 per CTA, so with few query rows (few CTAs) those rounds are the whole
+    // time.  Measured at 4 x 8 heads, split-KV against small-d: 64 x 1024 rows
+    // x keys 13.9 against 34.2 us, 128 x 2048 51.6 against about 69, 128 x 1024
+    // 50.8 against 34.4, 256 x 2048 98.8 against 66.7, 512 x 4096 268 against 131.
+    if (p.Tkv >= 1024 && (long long)p.Tq * 16 <= p.Tkv) return SDPA_PATH_SPLIT_KV;
     return SDPA_PATH_SMALL_D;
   }
   return SDPA_PATH_EXACT;

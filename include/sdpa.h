@@ -104,7 +104,7 @@ typedef enum {
   SDPA_PATH_SMALL_D = 3,   /* packed d=16 kernel, one query row per thread; bf16 */
   SDPA_PATH_SPLIT_KV = 4,  /* split-KV with in-kernel merge, short Tq / long Tkv; bf16, d=16;
                               tensor-core parts.  AUTO takes it when Tkv >= 1024 and
-                              Tq <= Tkv / 4 */
+                              Tq <= Tkv / 16 */
   SDPA_PATH_TC_PERSISTENT = 5 /* the tcgen05 kernel as one persistent CTA per SM walking many
                                  short problems (e.g. SAM's windowed attention: 14x14-token
                                  windows); bf16, d=64, no mask, rel-pos key-grid width 14 or 16

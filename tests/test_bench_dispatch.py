@@ -26,10 +26,10 @@ EXPECTED = {
 
 
 # head_dim-16 shapes on either side of the split-KV rule (Tkv >= 1024 and
-# Tq <= Tkv / 4), as (B, H, Tq, Tkv) -> family
-D16_RULE = [((4, 8, 8, 4096), "split_kv"), ((4, 8, 100, 8192), "split_kv"), ((4, 8, 256, 1024), "split_kv"),
-            ((4, 8, 257, 1024), "small_d"), ((4, 8, 8, 1023), "small_d"), ((4, 8, 4096, 8), "small_d"),
-            ((4, 8, 1024, 2048), "small_d")]
+# Tq <= Tkv / 16), as (B, H, Tq, Tkv) -> family
+D16_RULE = [((4, 8, 8, 4096), "split_kv"), ((4, 8, 100, 8192), "split_kv"), ((4, 8, 64, 1024), "split_kv"),
+            ((4, 8, 128, 2048), "split_kv"), ((4, 8, 129, 2048), "small_d"), ((4, 8, 128, 1024), "small_d"),
+            ((4, 8, 8, 1023), "small_d"), ((4, 8, 4096, 8), "small_d"), ((4, 8, 512, 4096), "small_d")]
 
 
 @pytest.mark.parametrize("shape,family", D16_RULE)

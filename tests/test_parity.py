@@ -75,6 +75,9 @@ CASES = [
        mask_neg_inf_frac=0.2, mask_heads=8, seed=47),
     S_("d16_packed2_sliding_odd_heads", BF16, 160, 3, 3, 16, 50, 16, mask_kind=W.MASK_SLIDING, window=9,
        offset=20, seed=48),
+    # the same packing on the tensor-core small-d kernel (64 keys or more):
+    # 8 heads of 13 rows per CTA, GQA, causal with an offset
+    S_("d16_packed8_mma_causal_gqa", BF16, 150, 8, 4, 13, 100, 16, mask_kind=W.MASK_CAUSAL, offset=60, seed=58),
     # rel-pos shapes the tensor-core path specialises (key-grid width 14/16/32/64)
     S_("relpos_bf16_d64_12x16", BF16, 2, 3, 3, 192, 192, 64, q_hw=(12, 16), k_hw=(12, 16), rel_std=0.5, seed=27),
     S_("relpos_bf16_d64_8x32", BF16, 1, 4, 2, 256, 256, 64, q_hw=(8, 32), k_hw=(8, 32), rel_std=0.5, seed=28),
