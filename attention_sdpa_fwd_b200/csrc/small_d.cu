@@ -2,30 +2,32 @@
 // issue "segment_anything: fuse attention ...": the TwoWayTransformer's
 // Attention, the same matmul/softmax/matmul without a bias; candle PR "SDPA
 // with Relative Positional Embeddings": head_dim 16 support and a packed
-// vector kernel for it).  At head_dim 16 a 128-row tensor-core tile would sit
-// mostly idle and the work is a stream over Q/O or K/V, so both kernels run
-// on CUDA cores and are shaped for HBM bandwidth:
+// vector kernel for it).  At head_dim 16 a 128-row tcgen05 tile would sit
+// mostly idle and the work is a stream over Q/O or K/V, so the kernels are
+// shaped for memory traffic, with the arithmetic on mma.sync tensor-core
+// tiles (16 rows x 8 or 16 keys) wherever there are enough keys to fill them:
 //
-//  * small_d_kernel: one thread per query row (16 values of q, the running
-//    max/sum and a 16-wide accumulator in registers), 128 consecutive rows of
-//    one (batch, head) per CTA so Q and O move as fully coalesced 32-byte
-//    rows.  K/V of the kv head stream through shared memory in chunks as fp32
-//    and are read by every thread as broadcasts.  Used when there are many
-//    query rows (image->token: 4096 rows against 8 keys; self-attention).
+//  * small_d_kernel / small_d_mma_kernel: one thread per query row for the
+//    global traffic (a 32-byte Q row in, an O row out), 128 consecutive rows
+//    of one (batch, head) per CTA -- or of several heads when the query axis
+//    is short -- and K/V rounds staged in shared memory.  The scalar kernel
+//    serves short key axes (image->token: 4096 rows against 8 keys); from 64
+//    keys on, the tensor-core instance.
 //
-//  * split_kv_kernel: few query rows against a long key axis (token->image: 8
-//    rows against 4096 keys).  The key axis of every (batch, head) is split
-//    over enough CTAs to cover the SMs; each CTA stages its K/V chunk in
-//    shared memory, one warp per query row runs the online softmax over the
-//    chunk (lanes stride the keys), and writes (m, l, unnormalised O) for its
-//    part.  The last CTA of a (batch, head) to finish, detected with an
-//    atomic ticket, merges the parts: O = sum_k 2^(m_k-M) O_k / sum_k 2^(m_k-M) l_k.
-//    When the key axis fits in 8 parts, split_kv_cluster_kernel does the
-//    same with the parts in one thread-block cluster, merged through
-//    distributed shared memory instead of a global workspace.
+//  * split_kv_kernel: few query rows against a long key axis.  The key axis
+//    of every (batch, head) is split over enough CTAs to cover the SMs; each
+//    CTA stages its K/V part, every warp computes the partial (m, l,
+//    unnormalised O) of each row over its slice of the keys on the tensor
+//    cores, the warps' partials merge in the CTA and go to a workspace, and
+//    the last CTA of a (batch, head) to finish, detected with an atomic
+//    ticket, merges the parts: O = sum_k 2^(m_k-M) O_k / sum_k 2^(m_k-M) l_k.
+//    When the key axis fits in 8 parts (token->image: 8 rows against 4096
+//    keys), split_kv_cluster_kernel does the same with the parts in one
+//    thread-block cluster, merged through distributed shared memory instead
+//    of a global workspace.
 //
-// Both take every mask kind and GQA; neither takes the rel-pos bias (the
-// exact kernel does).
+// All take every mask kind and GQA; none takes the rel-pos bias (the exact
+// kernel does).
 #include <math.h>
 
 #include <mutex>
