@@ -91,6 +91,8 @@ struct TcArgs {
   int n_full;    // units taken whole, first in launch order
   int n_split;   // parts per split unit (1 = no split units)
   int reverse_q; // take query blocks last-first (causal: the longest rows start first)
+  int head_fast; // number units head-fastest (a mask tensor shared by every head: the heads of a
+                 // query block run together and read its mask rows once from DRAM)
   float* ws_o;   // [split units][n_split][D/4][256] float4: unnormalised partial outputs
   float2* ws_ml; // [split units][n_split][256] (running max in log2 units, sum)
   int* ws_cnt;   // [split units] arrival counters, zero between launches
@@ -191,9 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     unit = args.n_full + i / nsplit;
     sidx = i - (i / nsplit) * nsplit;
   }
-  const int qraw = unit % args.nqblk;
+  const int qraw = args.head_fast ? (unit / args.Hq) % args.nqblk : unit % args.nqblk;
   const int qblk = args.reverse_q ? args.nqblk - 1 - qraw : qraw;
-  const int h = (unit / args.nqblk) % args.Hq;
+  const int h = args.head_fast ? unit % args.Hq : (unit / args.nqblk) % args.Hq;
   const int b = unit / (args.nqblk * args.Hq);
   const int hk = h / args.group;
   const int q0 = qblk * 2 * kRowsPerTile;
@@ -320,10 +322,13 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       int m_issued = 0;
       auto load_m = [&](int jj) {
         if constexpr (kMaskTma) {
+          // both query tiles' stages free first, then both loads: a wait that
+          // gives up leaves no load of this key tile in flight
           const int s = jj & 1, use = jj >> 1;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (use > 0) ok = mbar_wait(&m_empty[2 * t + s], (use - 1) & 1, abort_v, args.err);
-            if (!ok) return;
+          for (int t = 0; t < 2 && ok && use > 0; ++t)
+            ok = mbar_wait(&m_empty[2 * t + s], (use - 1) & 1, abort_v, args.err);
+          if (!ok) return;
+          for (int t = 0; t < 2; ++t) {
             mbar_expect_tx(&m_full[2 * t + s], L::kMaskBytes);
             tma_load_4d(sMask + (2 * t + s) * L::kMaskBytes, &args.tm, &m_full[2 * t + s], (j_begin + jj) * BN,
                         q0 + t * kRowsPerTile, args.msh ? h : 0, args.msb ? b : 0);
@@ -1125,6 +1130,9 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   a.nqblk = nqblk;
   // causal: query blocks with the most key tiles first, so the short ones fill the tail
   a.reverse_q = (mk == TC_RANGE && p.mask_kind == SDPA_MASK_CAUSAL) ? 1 : 0;
+  // a float / bool mask tensor broadcast over heads: every head of a query
+  // block reads the same mask rows, so those heads run side by side
+  a.head_fast = ((mk == TC_FLOAT || mk == TC_BOOL) && p.msh == 0 && p.Hq > 1) ? 1 : 0;
   const long long units = nblk_of(p, nqblk);
   const long long n_split_units = units - a.n_full;
   if (n_split_units > 0) {
