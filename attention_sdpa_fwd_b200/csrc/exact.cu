@@ -120,13 +120,15 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     l = l * corr + psum;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] *= corr;
-    // the value sum over the chunk's keys, eight at a time: the eight V loads
-    // go out together, then the eight FMAs (one round trip per eight keys)
+    // the value sum over the chunk's keys, KB at a time: the KB V loads go
+    // out together, then the FMAs (one round trip per KB keys; 16 when a lane
+    // owns one column)
+    constexpr int KB = CPL == 1 ? 16 : 8;
     const int nk = (int)((hi - j0) < 32 ? (hi - j0) : 32);
-    for (int t0 = 0; t0 < nk; t0 += 8) {
-      float pt[8], vv[8][CPL];
+    for (int t0 = 0; t0 < nk; t0 += KB) {
+      float pt[KB], vv[KB][CPL];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < KB; ++u) {
         const int t = t0 + u;  // < 32
         pt[u] = __shfl_sync(0xffffffffu, pj, t);
         const bool live = t < nk && owns_cols && dcheck_kv(p, b, hk, j0 + t);
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
         for (int c = 0; c < CPL; ++c) vv[u][c] = live ? to_f32(vr[c]) : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < KB; ++u)
 #pragma unroll
         for (int c = 0; c < CPL; ++c) acc[c] = fmaf(pt[u], vv[u][c], acc[c]);
     }
