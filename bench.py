@@ -396,7 +396,7 @@ def time_pinned_copies(device, h2d_bytes: int, d2h_bytes: int, reps: int = 10):
     return up_ms, down_ms
 
 
-# What bounds each workload's kernel (SURVEY-style work counts live in
+# What bounds each workload's kernel (the algorithmic work counts live in
 # workloads.Spec.flops / bytes): the dense contractions run against the bf16
 # tensor peak, the streaming shapes against HBM bandwidth, and the two tiny
 # problems (33 KB) are latency-bound and reported in microseconds only.
