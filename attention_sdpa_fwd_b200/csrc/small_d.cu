@@ -688,22 +688,31 @@ __global__ void __launch_bounds__(kSplitThreads, 3) split_kv_kernel(SplitArgs a)
 // thread-block cluster: each CTA leaves its partial (O, m, l) per query row
 // in its own shared memory, and the parts merge through distributed shared
 // memory -- no global workspace, fence or ticket, so the whole forward is one
-// pass over K and V.  Used when the key axis fits in 8 parts of at most 512
-// keys.  Inside a part, K and V are staged as bf16 with 16-byte loads (two
-// keys per thread), and warp w takes 64 of the keys: for every 16-row tile of
-// query rows, S = Q K^T, the softmax over its 64 keys and O = P V run on the
-// tensor cores (mma.sync).  The warps' partials merge in the CTA, the CTAs'
-// through the cluster.
-constexpr int kClusterMax = 8;      // portable cluster size
-constexpr int kClusterChunk = 512;  // keys per CTA (at most)
-constexpr int kWarpKeys = kClusterChunk / (kSplitThreads / 32);  // 64 keys per warp
+// pass over K and V.  Used when the key axis fits in the cluster's parts
+// (4096 keys).  Inside a part, K and V are staged as bf16 with 16-byte loads
+// (CHUNK / 256 keys per thread), and each warp takes CHUNK / 8 of the keys:
+// for every 16-row tile of query rows, S = Q K^T, the softmax over its keys
+// and O = P V run on the tensor cores (mma.sync).  The warps' partials merge
+// in the CTA, the CTAs' through the cluster.  Two sizes: 8 parts of 512 keys,
+// and 4 parts of 1024 keys for grids beyond one wave of two CTAs per SM, where
+// fewer and larger CTAs spread their fixed costs over more keys (token->image
+// at batch 128: 128 against 187 us; at batch 4: 8.2 against 7.5 us).
+constexpr int kClusterKeys = 4096;  // keys a cluster covers (at most)
 constexpr int kRowsMax = 64;        // query rows the partial areas hold
-// dynamic shared memory: K and V (bf16 rows), Q rows, the warps' partials,
-// the CTA's partials
-constexpr int kClK = 0, kClV = kClusterChunk * 32, kClQ = 2 * kClusterChunk * 32;
-constexpr int kClWarp = kClQ + kRowsMax * 32;
-constexpr int kClPart = kClWarp + (kSplitThreads / 32) * kRowsMax * kPartStride * 4;
-constexpr int kClBytes = kClPart + kRowsMax * kPartStride * 4;
+
+template <int NCL>
+struct ClLayout {
+  static constexpr int kChunk = kClusterKeys / NCL;                 // keys per CTA (at most)
+  static constexpr int kWarpKeys = kChunk / (kSplitThreads / 32);   // keys per warp
+  static constexpr int kKeysPerThread = kChunk / kSplitThreads;
+  // dynamic shared memory: K and V (bf16 rows), Q rows, the warps' partials,
+  // the CTA's partials
+  static constexpr int kK = 0, kV = kChunk * 32, kQ = 2 * kChunk * 32;
+  static constexpr int kWarp = kQ + kRowsMax * 32;
+  static constexpr int kPart = kWarp + (kSplitThreads / 32) * kRowsMax * kPartStride * 4;
+  static constexpr int kBytes = kPart + kRowsMax * kPartStride * 4;
+  static_assert(kChunk % kSplitThreads == 0 && kWarpKeys % 16 == 0, "whole keys per thread, 16-key tiles");
+};
 
 struct ClusterArgs {
   Params p;
@@ -711,15 +720,17 @@ struct ClusterArgs {
   int chunk;  // keys per part
 };
 
+template <int NCL>
 __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(ClusterArgs a) {
   namespace cg = cooperative_groups;
+  using CL = ClLayout<NCL>;
   const Params& p = a.p;
   constexpr int kWarps = kSplitThreads / 32;
   extern __shared__ __align__(128) uint8_t cl_smem[];
-  float* warp_s = reinterpret_cast<float*>(cl_smem + kClWarp);  // [kWarps][kRowsMax][kPartStride]
-  float* part_s = reinterpret_cast<float*>(cl_smem + kClPart);  // [kRowsMax][kPartStride], read by the cluster
-  const uint32_t k_s = sm100::smem_u32(cl_smem + kClK), v_s = sm100::smem_u32(cl_smem + kClV);
-  const uint32_t q_s = sm100::smem_u32(cl_smem + kClQ);
+  float* warp_s = reinterpret_cast<float*>(cl_smem + CL::kWarp);  // [kWarps][kRowsMax][kPartStride]
+  float* part_s = reinterpret_cast<float*>(cl_smem + CL::kPart);  // [kRowsMax][kPartStride], read by the cluster
+  const uint32_t k_s = sm100::smem_u32(cl_smem + CL::kK), v_s = sm100::smem_u32(cl_smem + CL::kV);
+  const uint32_t q_s = sm100::smem_u32(cl_smem + CL::kQ);
   cg::cluster_group cluster = cg::this_cluster();
   const int part = (int)cluster.block_rank(), h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.group;
@@ -729,12 +740,12 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mrows = (p.Tq + 15) & ~15;  // query rows rounded up to whole 16-row tiles
   {
-    // stage K and V rows tid and tid + 256 (zeros past the part) and Q rows
+    // stage K and V rows tid, tid + 256, ... (zeros past the part) and Q rows
     // (zeros past Tq), all loads issued before the first store
-    static_assert(kClusterChunk == 2 * kSplitThreads, "two keys per thread");
-    uint4 kv[2][4], qv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    constexpr int KPT = CL::kKeysPerThread;
+    uint4 kv[KPT][4], qv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < KPT; ++u) {
       const int tk = tid + u * kSplitThreads;
       kv[u][0] = kv[u][1] = kv[u][2] = kv[u][3] = make_uint4(0, 0, 0, 0);
       if (tk < n && dcheck_kv(p, b, hk, j0 + tk)) {
@@ -752,24 +763,24 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
       qv[1] = __ldg(qr + 1);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < KPT; ++u) {
       const int tk = tid + u * kSplitThreads;
-      *reinterpret_cast<uint4*>(cl_smem + kClK + sw32(tk, 0)) = kv[u][0];
-      *reinterpret_cast<uint4*>(cl_smem + kClK + sw32(tk, 1)) = kv[u][1];
-      *reinterpret_cast<uint4*>(cl_smem + kClV + sw32(tk, 0)) = kv[u][2];
-      *reinterpret_cast<uint4*>(cl_smem + kClV + sw32(tk, 1)) = kv[u][3];
+      *reinterpret_cast<uint4*>(cl_smem + CL::kK + sw32(tk, 0)) = kv[u][0];
+      *reinterpret_cast<uint4*>(cl_smem + CL::kK + sw32(tk, 1)) = kv[u][1];
+      *reinterpret_cast<uint4*>(cl_smem + CL::kV + sw32(tk, 0)) = kv[u][2];
+      *reinterpret_cast<uint4*>(cl_smem + CL::kV + sw32(tk, 1)) = kv[u][3];
     }
     if (tid < mrows) {
-      *reinterpret_cast<uint4*>(cl_smem + kClQ + sw32(tid, 0)) = qv[0];
-      *reinterpret_cast<uint4*>(cl_smem + kClQ + sw32(tid, 1)) = qv[1];
+      *reinterpret_cast<uint4*>(cl_smem + CL::kQ + sw32(tid, 0)) = qv[0];
+      *reinterpret_cast<uint4*>(cl_smem + CL::kQ + sw32(tid, 1)) = qv[1];
     }
   }
   __syncthreads();
   const float sl = p.scale * kLog2e;
-  const int kw0 = warp * kWarpKeys;  // this warp's keys within the part: [kw0, kw0 + 64)
+  const int kw0 = warp * CL::kWarpKeys;  // this warp's keys within the part
   float* wp = warp_s + warp * kRowsMax * kPartStride;
   for (int row0 = 0; row0 < p.Tq; row0 += 16)
-    warp_slice_partial<kWarpKeys / 16>(p, b, h, q_s, row0, k_s, v_s, kw0, n, j0, row0, wp + row0 * kPartStride, lane,
+    warp_slice_partial<CL::kWarpKeys / 16>(p, b, h, q_s, row0, k_s, v_s, kw0, n, j0, row0, wp + row0 * kPartStride, lane,
                                        sl);
   __syncthreads();
   // the CTA's partial of row i from its warps' (warp i % 8 combines row i)
@@ -803,7 +814,7 @@ __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(Clus
     // lane c (< 16) sums column c over the parts
     float num = 0.f;
 #pragma unroll
-    for (int k = 0; k < kClusterMax; ++k) {
+    for (int k = 0; k < NCL; ++k) {
       const float w_k = __shfl_sync(0xffffffffu, wk, k);
       if (k < a.ncl && lane < D16 && w_k > 0.f)
         num = fmaf(w_k, cluster.map_shared_rank(part_s, k)[i * kPartStride + lane], num);
@@ -905,34 +916,42 @@ cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream
   return cudaGetLastError();
 }
 
+template <int NCL>
+static cudaError_t launch_cluster(const Params& p, cudaStream_t stream) {
+  using CL = ClLayout<NCL>;
+  ClusterArgs a;
+  a.p = p;
+  a.ncl = NCL;
+  a.chunk = (p.Tkv + NCL - 1) / NCL;
+  const size_t smem = (size_t)CL::kBytes;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] {
+    attr = cudaFuncSetAttribute(split_kv_cluster_kernel<NCL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (attr != cudaSuccess) return attr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)NCL, (unsigned)p.Hq, (unsigned)p.B);
+  cfg.blockDim = dim3(kSplitThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)NCL;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, split_kv_cluster_kernel<NCL>, a);
+}
+
 cudaError_t launch_split_kv(const Params& p, cudaStream_t stream) {
-  // one cluster of up to 8 parts per (batch, head) when the key axis fits
-  if (p.Tq <= kRowsMax && p.Tkv >= 1 && p.Tkv <= (long long)kClusterMax * kClusterChunk && p.B <= 65535 &&
-      p.Hq <= 65535) {
-    ClusterArgs a;
-    a.p = p;
-    a.ncl = kClusterMax;
-    a.chunk = (p.Tkv + kClusterMax - 1) / kClusterMax;
-    const size_t smem = (size_t)kClBytes;
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [&] {
-      attr = cudaFuncSetAttribute(split_kv_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    });
-    if (attr != cudaSuccess) return attr;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)a.ncl, (unsigned)p.Hq, (unsigned)p.B);
-    cfg.blockDim = dim3(kSplitThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = (unsigned)a.ncl;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, split_kv_cluster_kernel, a);
+  // one cluster of parts per (batch, head) when the key axis fits: 8 parts,
+  // or 4 larger ones once 8-part clusters would not fit one wave of two CTAs
+  // per SM
+  if (p.Tq <= kRowsMax && p.Tkv >= 1 && p.Tkv <= (long long)kClusterKeys && p.B <= 65535 && p.Hq <= 65535) {
+    if ((long long)p.B * p.Hq * 8 > 2LL * num_sms()) return launch_cluster<4>(p, stream);
+    return launch_cluster<8>(p, stream);
   }
   size_t cb = 0, db = 0;
   split_kv_workspace_bytes(p, &cb, &db);

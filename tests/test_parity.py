@@ -75,6 +75,11 @@ CASES = [
        mask_neg_inf_frac=0.2, mask_heads=8, seed=47),
     S_("d16_packed2_sliding_odd_heads", BF16, 160, 3, 3, 16, 50, 16, mask_kind=W.MASK_SLIDING, window=9,
        offset=20, seed=48),
+    # enough (batch, head) pairs for the split-KV clusters of 4 larger parts
+    # (more than one wave of 8-part clusters): plain, and a float mask per head
+    S_("d16_cluster4_cross", BF16, 10, 4, 2, 9, 3000, 16, seed=59),
+    S_("d16_cluster4_float_mask", BF16, 13, 3, 3, 20, 1234, 16, mask_kind=W.MASK_FLOAT, mask_std=1.0,
+       mask_neg_inf_frac=0.2, mask_heads=3, seed=60),
     # the same packing on the tensor-core small-d kernel (64 keys or more):
     # 8 heads of 13 rows per CTA, GQA, causal with an offset
     S_("d16_packed8_mma_causal_gqa", BF16, 150, 8, 4, 13, 100, 16, mask_kind=W.MASK_CAUSAL, offset=60, seed=58),
