@@ -183,6 +183,21 @@ SPECS: Dict[str, Spec] = {
                            mask_heads=1),
 }
 
+# Shapes outside the benchmark, for the ncu evidence of kernels no benchmark
+# workload reaches: head_dim 16 with long key axes, on the tensor-core small-d
+# kernel (1024 query rows against 2048 keys) and on the global-workspace
+# split-KV kernel (8 rows against 16384 keys).
+EXTRA_SPECS: Dict[str, Spec] = {
+    "d16_long_self": Spec("d16_long_self", BF16, 4, 8, 8, 1024, 2048, 16, 0.25, seed=3),
+    "d16_very_long_keys": Spec("d16_very_long_keys", BF16, 4, 8, 8, 8, 16384, 16, 0.25, seed=3),
+}
+
+
+def spec_named(name: str) -> Spec:
+    """A benchmark workload, or one of the extra profiling shapes."""
+    return SPECS[name] if name in SPECS else EXTRA_SPECS[name]
+
+
 # Bias-dominated companions: with these the bias decides the scores, so a
 # missing or misindexed bias fails every gate.
 STRONG_SPECS: Dict[str, Spec] = {

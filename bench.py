@@ -538,7 +538,7 @@ def run_profile_launches(args):
     torch.cuda.set_device(device)
     import attention_sdpa_fwd_b200 as S
     S.lib()
-    spec = W.SPECS[args.workload]
+    spec = W.spec_named(args.workload)
     spec = W.scaled(spec, B=args.batch if args.batch > 0 else spec.B * args.batch_mult)
     st = make_device_sets(spec, device, 1, seed_base=spec.seed)[0]
     stream = torch.cuda.current_stream(device)
@@ -566,7 +566,7 @@ def run_ours(args):
         pass
     S.lib()  # fails loudly if the extension is missing
     peaks, peaks_src = load_peaks()
-    spec = W.SPECS[args.workload]
+    spec = W.spec_named(args.workload)
 
     sampler = ClockSampler(torch.cuda.current_device() if ws == 1 else local)
     sampler.start()
@@ -653,7 +653,7 @@ def run_reference(args):
     ws, rank, local = dist_env()
     if rank != 0:
         return
-    spec = W.SPECS[args.workload]
+    spec = W.spec_named(args.workload)
     vals = []
     info = None
     # about 150 s of oracle work in all, whatever --steps / --warmup ask for
@@ -683,7 +683,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="sam_global", choices=sorted(W.SPECS))
+    ap.add_argument("--workload", default="sam_global", choices=sorted(W.SPECS) + sorted(W.EXTRA_SPECS))
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload table (every benchmark workload timed through AUTO)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
