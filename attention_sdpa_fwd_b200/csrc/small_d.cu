@@ -279,8 +279,18 @@ __device__ __forceinline__ void warp_slice_partial(const Params& p, int b, int h
       mma16816(x[c][u], qa, kf[2 * u], kf[2 * u + 1]);
     }
   }
-  // scores in log2 units with the mask; absent keys and rows past Tq score -inf
+  // scores in log2 units with the mask; absent keys and rows past Tq score
+  // -inf (a warp slice of present keys without a mask: the scale and the row test)
   const long long mrow_base = (long long)b * p.msb + (long long)h * p.msh;
+  if (p.mask_kind == SDPA_MASK_NONE && key0 + 16 * NT <= n) {
+    const bool ok0 = row0 + g < p.Tq, ok1 = row0 + g + 8 < p.Tq;
+#pragma unroll
+    for (int c = 0; c < NT; ++c)
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[c][u][e] = ((e >> 1) ? ok1 : ok0) ? x[c][u][e] * sl : -INFINITY;
+  } else
 #pragma unroll
   for (int c = 0; c < NT; ++c)
 #pragma unroll
@@ -485,6 +495,13 @@ __global__ void __launch_bounds__(kRowsPerCta, MASKED ? 4 : 6) small_d_mma_kerne
         mma16816(x[0], qa[m], kf[0], kf[1]);
         mma16816(x[1], qa[m], kf[2], kf[3]);
         const long long mrow_base = (long long)b * p.msb + (long long)hm[m] * p.msh;
+        if (!MASKED && k0 + 16 <= n && row0[m] + 16 <= p.Tq) {
+          // a whole tile of present keys and rows: only the scale
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[u][e] *= sl;
+        } else
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
