@@ -552,24 +552,42 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       if (ok) {
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
+          // key-grid coordinate k of this row is reached through table row
+          // (= projection column) base - k, 0 <= k < nk
           const int base_idx = w == 0 ? qh + kh_n - 1 : qw + KW - 1;
-          const int nk = w == 0 ? kh_n : KW;
+          const unsigned nk = w == 0 ? kh_n : KW;
+          // the columns any row of this warp takes (when a warp shares one
+          // query-grid row and spans 32 grid columns, at most three of the four
+          // 32-column chunks), all loaded before one wait
+          const int c_lo = __reduce_min_sync(0xffffffffu, base_idx) - (int)nk + 1;
+          const int c_hi = __reduce_max_sync(0xffffffffu, base_idx);
+          uint32_t r[4][32];
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            if (c0 < args.rel_n) {
-              uint32_t r[32];
-              tmem_ld32(tbase + lane_off + t * 256 + w * 128 + c0, r);
-              tmem_wait_ld();
+          for (int j = 0; j < 4; ++j)
+            if (32 * j < args.rel_n && 32 * j + 31 >= c_lo && 32 * j <= c_hi)
+              tmem_ld32(tbase + lane_off + t * 256 + w * 128 + 32 * j, r[j]);
+          tmem_wait_ld();
+          if (w == 1) {
+            // every projection column this thread reads is in registers: the
+            // columns may take Q.K^T of the first key tile while the scatter runs
+            tc_fence_before();
+            mbar_arrive(rel_read);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (32 * j < args.rel_n && 32 * j + 31 >= c_lo && 32 * j <= c_hi) {
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
-                const int k = base_idx - (c0 + i);  // key-grid coordinate reached through table row c0+i
-                if (k >= 0 && k < nk && dcheck_idx(args.err, k, w == 0 ? kRelHMax : KW)) {
-                  const float val = __uint_as_float(r[i]) * kLog2e;
+                const int k = base_idx - (32 * j + i);
+                if ((unsigned)k < nk && dcheck_idx(args.err, k, w == 0 ? kRelHMax : KW)) {
+                  const float val = __uint_as_float(r[j][i]) * kLog2e;
                   if (w == 1 && kRwInSmem)
-                    // this row's slice, float4 groups XOR-swizzled by row: the
-                    // loop reads it as float4 without bank conflicts (and so
-                    // does this scatter when the query and key grids have equal width)
-                    relw_s[row * KW + ((((k >> 2) ^ (row & kRwSwz)) << 2) | (k & 3))] = val;
+                    // this row's slice, float4 groups XOR-swizzled by row (float4
+                    // group g at g ^ (row & kRwSwz), i.e. element k at
+                    // k ^ ((row & kRwSwz) << 2)): the loop reads it as float4
+                    // without bank conflicts, and so does this scatter when the
+                    // query and key grids have equal width
+                    relw_s[row * KW + (k ^ ((row & kRwSwz) << 2))] = val;
                   else
                     // [k][256]: consecutive rows hit consecutive banks whatever k is
                     (w == 0 ? relh_s : relw_s)[k * 256 + row] = val;
@@ -578,10 +596,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
             }
           }
         }
+      } else {
+        tc_fence_before();
+        mbar_arrive(rel_read);
       }
-      // every thread reads back only what it wrote itself: no CTA barrier needed
-      tc_fence_before();
-      mbar_arrive(rel_read);
+      // every thread reads back only what it wrote itself: no CTA barrier is
+      // needed before the loop
     }
 
     // per-row visible key range (causal / sliding)
