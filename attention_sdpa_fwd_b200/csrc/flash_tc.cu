@@ -550,7 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       const int qw_n = args.qw_n, kh_n = args.kh_n;
       const int qh = (int)(qi / qw_n), qw = (int)(qi % qw_n);
       if (ok) {
-#pragma unroll
+        // rolled over w and the chunks: this code runs once per CTA, from a
+        // cold instruction cache
+#pragma unroll 1
         for (int w = 0; w < 2; ++w) {
           // key-grid coordinate k of this row is reached through table row
           // (= projection column) base - k, 0 <= k < nk
@@ -558,30 +560,24 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
           const unsigned nk = w == 0 ? kh_n : KW;
           // the columns any row of this warp takes (when a warp shares one
           // query-grid row and spans 32 grid columns, at most three of the four
-          // 32-column chunks), all loaded before one wait
+          // 32-column chunks)
           const int c_lo = __reduce_min_sync(0xffffffffu, base_idx) - (int)nk + 1;
           const int c_hi = __reduce_max_sync(0xffffffffu, base_idx);
-          uint32_t r[4][32];
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (32 * j < args.rel_n && 32 * j + 31 >= c_lo && 32 * j <= c_hi)
-              tmem_ld32(tbase + lane_off + t * 256 + w * 128 + 32 * j, r[j]);
-          tmem_wait_ld();
-          if (w == 1) {
-            // every projection column this thread reads is in registers: the
-            // columns may take Q.K^T of the first key tile while the scatter runs
-            tc_fence_before();
-            mbar_arrive(rel_read);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (32 * j < args.rel_n && 32 * j + 31 >= c_lo && 32 * j <= c_hi) {
+          float* dst_h = w == 0 ? relh_s : relw_s;
+          const bool swz = w == 1 && kRwInSmem;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            if (c0 < args.rel_n && c0 + 31 >= c_lo && c0 <= c_hi) {
+              uint32_t r[32];
+              tmem_ld32(tbase + lane_off + t * 256 + w * 128 + c0, r);
+              tmem_wait_ld();
+              const int kb = base_idx - c0;
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
-                const int k = base_idx - (32 * j + i);
+                const int k = kb - i;
                 if ((unsigned)k < nk && dcheck_idx(args.err, k, w == 0 ? kRelHMax : KW)) {
-                  const float val = __uint_as_float(r[j][i]) * kLog2e;
-                  if (w == 1 && kRwInSmem)
+                  const float val = __uint_as_float(r[i]) * kLog2e;
+                  if (swz)
                     // this row's slice, float4 groups XOR-swizzled by row (float4
                     // group g at g ^ (row & kRwSwz), i.e. element k at
                     // k ^ ((row & kRwSwz) << 2)): the loop reads it as float4
@@ -590,18 +586,17 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
                     relw_s[row * KW + (k ^ ((row & kRwSwz) << 2))] = val;
                   else
                     // [k][256]: consecutive rows hit consecutive banks whatever k is
-                    (w == 0 ? relh_s : relw_s)[k * 256 + row] = val;
+                    dst_h[k * 256 + row] = val;
                 }
               }
             }
           }
         }
-      } else {
-        tc_fence_before();
-        mbar_arrive(rel_read);
       }
       // every thread reads back only what it wrote itself: no CTA barrier is
       // needed before the loop
+      tc_fence_before();
+      mbar_arrive(rel_read);
     }
 
     // per-row visible key range (causal / sliding)
