@@ -141,6 +141,29 @@ int tc_persist_check(const Params& p, sdpa_dtype_t dtype);
 bool tc_persist_preferred(const Params& p);
 cudaError_t launch_tc_persist(const Params& p, cudaStream_t stream);
 
+// Division by a divisor d >= 1 fixed at launch, as a multiply-high, an add
+// and a shift (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", 1994, section 4, unsigned division by a run-time invariant
+// divisor): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1 (which
+// fits in 32 bits), n / d = (umulhi(m, n) + n) >> l for every 32-bit unsigned
+// n, the sum taken in 64 bits.  The kernels decode their work unit with it:
+// a generic 32-bit division is a long dependent chain at the head of every CTA.
+struct FastDiv {
+  uint32_t d, m, l;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d < 1 ? 1 : d;
+  uint32_t l = 0;
+  while ((1ull << l) < f.d) ++l;
+  f.l = l;
+  f.m = (uint32_t)((((1ull << 32) * ((1ull << l) - f.d)) / f.d) + 1);
+  return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (uint32_t)(((uint64_t)__umulhi(f.m, n) + n) >> f.l);
+}
+
 // Parts sdpa_merge combines at most.
 constexpr int kMaxMergeParts = 16;
 cudaError_t launch_merge(const void* const* outs, const float* const* lses, int n, void* out, float* lse,

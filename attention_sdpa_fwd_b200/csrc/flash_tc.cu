@@ -97,6 +97,8 @@ struct TcArgs {
   float2* ws_ml; // [split units][n_split][256] (running max in log2 units, sum)
   int* ws_cnt;   // [split units] arrival counters, zero between launches
   int* err;
+  // the divisors of the unit decode and of the query grid, as FastDiv
+  FastDiv fd_split, fd_hq, fd_nqblk, fd_group, fd_qw;
 };
 
 template <int D, int BN, int KW, int NS, int MT = 0>  // MT: bytes per mask element (0: no mask tiles)
@@ -190,14 +192,25 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   } else {
     const int i = blockIdx.x - args.n_full;
     nsplit = args.n_split;
-    unit = args.n_full + i / nsplit;
-    sidx = i - (i / nsplit) * nsplit;
+    const int pu = (int)fdiv((uint32_t)i, args.fd_split);
+    unit = args.n_full + pu;
+    sidx = i - pu * nsplit;
   }
-  const int qraw = args.head_fast ? (unit / args.Hq) % args.nqblk : unit % args.nqblk;
+  // unit = (b * Hq + h) * nqblk + qraw, or (b * nqblk + qraw) * Hq + h head-fastest
+  int qraw, h, b;
+  if (args.head_fast) {
+    const int u1 = (int)fdiv((uint32_t)unit, args.fd_hq);
+    h = unit - u1 * args.Hq;
+    b = (int)fdiv((uint32_t)u1, args.fd_nqblk);
+    qraw = u1 - b * args.nqblk;
+  } else {
+    const int u1 = (int)fdiv((uint32_t)unit, args.fd_nqblk);
+    qraw = unit - u1 * args.nqblk;
+    b = (int)fdiv((uint32_t)u1, args.fd_hq);
+    h = u1 - b * args.Hq;
+  }
   const int qblk = args.reverse_q ? args.nqblk - 1 - qraw : qraw;
-  const int h = args.head_fast ? unit % args.Hq : (unit / args.nqblk) % args.Hq;
-  const int b = unit / (args.nqblk * args.Hq);
-  const int hk = h / args.group;
+  const int hk = (int)fdiv((uint32_t)h, args.fd_group);
   const int q0 = qblk * 2 * kRowsPerTile;
 
   // Key-tile range of the query block (causal / sliding skip whole tiles) ...
@@ -216,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     }
   }
   // ... and this CTA's share of it
-  const int j_begin = jb + (int)((long long)(je - jb) * sidx / nsplit);
-  const int j_end = jb + (int)((long long)(je - jb) * (sidx + 1) / nsplit);
+  const int j_begin = nsplit == 1 ? jb : jb + (int)fdiv((uint32_t)((je - jb) * sidx), args.fd_split);
+  const int j_end = nsplit == 1 ? je : jb + (int)fdiv((uint32_t)((je - jb) * (sidx + 1)), args.fd_split);
   const int n_tiles = j_end - j_begin;
   // debug builds: the unit and its share of key tiles lie inside the problem
   // (uniform over the CTA, so the whole CTA leaves before any barrier)
@@ -548,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
       ok = __all_sync(0xffffffffu, mbar_wait(rel_mma, 0, abort_v, args.err));
       tc_fence_after();
       const int qw_n = args.qw_n, kh_n = args.kh_n;
-      const int qh = (int)(qi / qw_n), qw = (int)(qi % qw_n);
+      const int qh = (int)fdiv((uint32_t)qi, args.fd_qw), qw = (int)qi - qh * qw_n;
       if (ok) {
         // rolled over w and the chunks: this code runs once per CTA, from a
         // cold instruction cache
@@ -1148,6 +1161,11 @@ cudaError_t launch_tc(const Params& p, cudaStream_t stream) {
   // a float / bool mask tensor broadcast over heads: every head of a query
   // block reads the same mask rows, so those heads run side by side
   a.head_fast = ((mk == TC_FLOAT || mk == TC_BOOL) && p.msh == 0 && p.Hq > 1) ? 1 : 0;
+  a.fd_split = make_fastdiv((uint32_t)a.n_split);
+  a.fd_hq = make_fastdiv((uint32_t)p.Hq);
+  a.fd_nqblk = make_fastdiv((uint32_t)nqblk);
+  a.fd_group = make_fastdiv((uint32_t)p.group);
+  a.fd_qw = make_fastdiv((uint32_t)p.qw_n);
   const long long units = nblk_of(p, nqblk);
   const long long n_split_units = units - a.n_full;
   if (n_split_units > 0) {
