@@ -79,6 +79,9 @@ struct PsArgs {
   int nqblk;   // 256-row query blocks per (batch, head)
   int units;   // nqblk * Hq * B
   int* err;
+  // the divisors of the unit decode, of the tile count and of the query grid,
+  // as FastDiv (the CTA count is the grid's, fixed at launch)
+  FastDiv fd_nqblk, fd_hq, fd_group, fd_nt, fd_qw, fd_grid;
 };
 
 template <int BN, int KW, int NS>
@@ -108,10 +111,10 @@ struct UnitPos {
 
 __device__ __forceinline__ UnitPos unit_pos(const PsArgs& a, int u) {
   UnitPos r;
-  const int bh = u / a.nqblk;
+  const int bh = (int)fdiv((uint32_t)u, a.fd_nqblk);
   r.q0 = (u - bh * a.nqblk) * 2 * kRows;
-  r.h = bh % a.Hq;
-  r.b = bh / a.Hq;
+  r.b = (int)fdiv((uint32_t)bh, a.fd_hq);
+  r.h = bh - r.b * a.Hq;
   return r;
 }
 
@@ -147,7 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int G = gridDim.x;
-  const int n_units = (int)blockIdx.x < args.units ? (args.units - (int)blockIdx.x + G - 1) / G : 0;
+  const int n_units =
+      (int)blockIdx.x < args.units ? (int)fdiv((uint32_t)(args.units - (int)blockIdx.x + G - 1), args.fd_grid) : 0;
   const int nt = (args.Tkv + BN - 1) / BN;
   const int total = n_units * nt;
 
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
       for (int t = 0; t < 2; ++t)
         tma_load_4d(sQ + t * L::kQBytes, &args.tq, &q_full[0], 0, u0.q0 + t * kRows, u0.h, u0.b);
       mbar_expect_tx(&k_full[0], L::kKVBytes);
-      tma_load_4d(sK, &args.tk, &k_full[0], 0, 0, u0.h / args.group, u0.b);
+      tma_load_4d(sK, &args.tk, &k_full[0], 0, 0, (int)fdiv((uint32_t)u0.h, args.fd_group), u0.b);
     }
   }
   if (warp == 9) {
@@ -203,13 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
           const int s = g % NS, use = g / NS;
           if (use > 0) ok = mbar_wait(is_k ? &k_empty[s] : &v_empty[s], (use - 1) & 1, abort_v, args.err);
           if (!ok) return;
-          const int it = g / nt;
+          const int it = (int)fdiv((uint32_t)g, args.fd_nt);
           const UnitPos u = unit_pos(args, blockIdx.x + it * G);
           const int key0 = (g - it * nt) * BN;
           uint64_t* bar = is_k ? &k_full[s] : &v_full[s];
           mbar_expect_tx(bar, L::kKVBytes);
           tma_load_4d((is_k ? sK : sV) + s * L::kKVBytes, is_k ? &args.tk : &args.tv, bar, 0, key0,
-                      u.h / args.group, u.b);
+                      (int)fdiv((uint32_t)u.h, args.fd_group), u.b);
           if (is_k) k_issued = g + 1; else v_issued = g + 1;
         };
         for (int g = 1; g < total && ok; ++g) {
@@ -312,10 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
           mma_commit_w(&k_empty[0]);
         }
         for (int g = 0; g < total && ok; ++g) {
-          const int it = g / nt, j = g - it * nt, s = g % NS;
+          const int it = (int)fdiv((uint32_t)g, args.fd_nt), j = g - it * nt, s = g % NS;
           const int g1 = g + 1;
           const bool more = g1 < total;
-          const int it1 = g1 / nt, j1 = g1 - it1 * nt, s1 = g1 % NS, qb1 = it1 & 1;
+          const int it1 = (int)fdiv((uint32_t)g1, args.fd_nt), j1 = g1 - it1 * nt, s1 = g1 % NS, qb1 = it1 & 1;
           if (more) {
             if (j1 == 0) ok = wait(&q_full[qb1], (it1 >> 1) & 1);
             if (ok) ok = wait(&k_full[s1], (g1 / NS) & 1);
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
         ok = __all_sync(0xffffffffu, mbar_wait(rel_mma, it & 1, abort_v, args.err));
         if (!ok) break;
         tc_fence_after();
-        const int qh = (int)(qi / args.qw_n), qw = (int)(qi % args.qw_n), kh_n = args.kh_n;
+        const int qh = (int)fdiv((uint32_t)qi, args.fd_qw), qw = (int)qi - qh * args.qw_n, kh_n = args.kh_n;
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           uint32_t r[32];
@@ -611,6 +615,12 @@ cudaError_t launch_tc_persist(const Params& p, cudaStream_t stream) {
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
   a.units = (int)units;
   const int grid = (int)(units < num_sms() ? units : num_sms());
+  a.fd_nqblk = make_fastdiv((uint32_t)a.nqblk);
+  a.fd_hq = make_fastdiv((uint32_t)p.Hq);
+  a.fd_group = make_fastdiv((uint32_t)p.group);
+  a.fd_nt = make_fastdiv((uint32_t)((p.Tkv + persist_bn(p) - 1) / persist_bn(p)));
+  a.fd_qw = make_fastdiv((uint32_t)p.qw_n);
+  a.fd_grid = make_fastdiv((uint32_t)(grid > 0 ? grid : 1));
   if (!p.use_rel) return launch_persist_one<128, 0, 4>(a, grid, stream);
   if (p.kw_n == 14) return launch_persist_one<112, 14, 4>(a, grid, stream);
   return launch_persist_one<128, 16, 3>(a, grid, stream);
