@@ -149,6 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  // programmatic dependent launch, as in the tensor-core kernel: nothing
+  // before grid_dep_wait() touches global memory
+  grid_dep_launch();
   const int G = gridDim.x;
   const int n_units =
       (int)blockIdx.x < args.units ? (int)fdiv((uint32_t)(args.units - (int)blockIdx.x + G - 1), args.fd_grid) : 0;
@@ -165,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
     mbar_init(&o_drained[0], 8);
     mbar_init(&o_drained[1], 8);
     fence_mbar_init();
+    grid_dep_wait();
     if (n_units > 0) {
       // the first unit's Q, the rel tables and K tile 0 go out before the
       // TMEM allocation and the CTA barrier
@@ -187,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_persist(const __grid_co
     tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
+  grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -547,8 +552,19 @@ cudaError_t launch_persist_one(const PsArgs& a, int grid, cudaStream_t stream) {
     if (attr_err == cudaSuccess && fa.numRegs != kRegsLaunch) attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(a);
-  return cudaGetLastError();
+  // programmatic serialization (the kernel waits for the previous grid before
+  // it touches global memory)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 bool al16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }

@@ -186,6 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  // Launched behind another grid (programmatic serialization), this CTA may
+  // start while that grid runs: everything before grid_dep_wait() touches
+  // only kernel parameters, shared memory and TMEM.  The next grid may be
+  // scheduled once every CTA of this one has started; its CTAs take SMs as
+  // this grid's leave and wait for its completion there.
+  grid_dep_launch();
   int unit, sidx = 0, nsplit = 1;  // sidx: which part of the unit's key range this CTA takes
   if ((int)blockIdx.x < args.n_full) {
     unit = blockIdx.x;
@@ -251,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     if constexpr (kMaskTma)
       for (int i = 0; i < 4; ++i) mbar_init(&m_empty[i], kRowsPerTile);
     fence_mbar_init();
+    grid_dep_wait();
     if (n_tiles > 0) {
       // Q (and the rel tables) and the first K tile go out before the TMEM
       // allocation and the CTA barrier, so their latency overlaps the setup
@@ -277,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
     tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
+  grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1010,8 +1018,20 @@ cudaError_t launch_one(const TcArgs& a, dim3 grid, cudaStream_t stream) {
     if (attr_err == cudaSuccess && fa.numRegs != kRegsLaunch) attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(a);
-  return cudaGetLastError();
+  // programmatic serialization: this grid's CTAs may be scheduled before the
+  // previous grid in the stream completes (the kernel waits for it before it
+  // touches global memory), hiding the launch gap between consecutive calls
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <int D, int BN, int KW, int NS>
