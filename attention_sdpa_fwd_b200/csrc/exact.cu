@@ -15,6 +15,8 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "pdl_launch.cuh"
+#include "sm100.cuh"
 
 namespace sdpa {
 namespace {
@@ -45,6 +47,10 @@ __device__ __forceinline__ float dot_any(const float* __restrict__ qs, const T* 
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
+  // launched behind the previous grid in the stream (programmatic
+  // serialization): wait for it before any global-memory access
+  sm100::grid_dep_launch();
+  sm100::grid_dep_wait();
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -164,8 +170,7 @@ cudaError_t launch_t(const Params& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   dim3 grid((unsigned)((p.Tq + kWarps - 1) / kWarps), (unsigned)p.Hq, (unsigned)p.B);
-  exact_kernel<T, D><<<grid, kWarps * 32, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_serialized(exact_kernel<T, D>, grid, dim3(kWarps * 32), smem, stream, p);
 }
 
 }  // namespace

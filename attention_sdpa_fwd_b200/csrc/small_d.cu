@@ -35,6 +35,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "pdl_launch.cuh"
 #include "sm100.cuh"
 
 namespace sdpa {
@@ -85,6 +86,10 @@ constexpr int kKeyChunk = 128;
 // 128 threads idle.  Each group stages its own head's keys, `rows` per
 // round, in its own slice of the shared K/V chunk.
 __global__ void __launch_bounds__(kRowsPerCta, 7) small_d_kernel(Params p, int hp_log2) {
+  // launched behind the previous grid in the stream (programmatic
+  // serialization): wait for it before any global-memory access
+  sm100::grid_dep_launch();
+  sm100::grid_dep_wait();
   __shared__ float4 sk[kKeyChunk][D16 / 4];  // every thread of a group reads the same key: broadcast
   __shared__ float4 sv[kKeyChunk][D16 / 4];
   const int rows = kRowsPerCta >> hp_log2;  // threads (query rows) per head
@@ -397,6 +402,8 @@ __device__ __forceinline__ void stsm_x4(uint32_t addr, const uint32_t (&r)[4]) {
 
 template <bool MASKED>
 __global__ void __launch_bounds__(kRowsPerCta, MASKED ? 4 : 6) small_d_mma_kernel(Params p, int hp_log2) {
+  sm100::grid_dep_launch();  // programmatic serialization when launched with it, as small_d_kernel
+  sm100::grid_dep_wait();
   __shared__ __align__(128) uint8_t sq[kRowsPerCta * 32];  // Q rows, then O rows (bf16, swizzled)
   __shared__ __align__(128) uint8_t sk[kRowsPerCta * 32];  // staged K rows
   __shared__ __align__(128) uint8_t sv[kRowsPerCta * 32];  // staged V rows
@@ -588,6 +595,8 @@ struct SplitArgs {
 constexpr int kWsRows = 32;  // query rows per block of the workspace kernel (two 16-row tiles)
 
 __global__ void __launch_bounds__(kSplitThreads, 3) split_kv_kernel(SplitArgs a) {
+  sm100::grid_dep_launch();  // programmatic serialization, as in small_d_kernel
+  sm100::grid_dep_wait();
   const Params& p = a.p;
   constexpr int kWarps = kSplitThreads / 32;
   static_assert(kSplitChunk == kSplitThreads && kSplitChunk == kWarps * 32, "a key per thread, 32 per warp");
@@ -739,6 +748,8 @@ struct ClusterArgs {
 
 template <int NCL>
 __global__ void __launch_bounds__(kSplitThreads, 2) split_kv_cluster_kernel(ClusterArgs a) {
+  sm100::grid_dep_launch();  // programmatic serialization, as in small_d_kernel
+  sm100::grid_dep_wait();
   namespace cg = cooperative_groups;
   using CL = ClLayout<NCL>;
   const Params& p = a.p;
@@ -883,9 +894,13 @@ cudaError_t launch_small_d(const Params& p, cudaStream_t stream) {
   const int hp = mma ? min(small_d_pack_log2(p), 3) : small_d_pack_log2(p);  // >= 16 rows a head on the tensor cores
   const int rows = kRowsPerCta >> hp;
   dim3 grid((unsigned)((p.Tq + rows - 1) / rows), (unsigned)((p.Hq + (1 << hp) - 1) >> hp), (unsigned)p.B);
-  if (!mma)
-    small_d_kernel<<<grid, kRowsPerCta, 0, stream>>>(p, hp);
-  else if (p.mask_kind == SDPA_MASK_NONE)
+  if (!mma) return launch_serialized(small_d_kernel, grid, dim3(kRowsPerCta), 0, stream, p, hp);
+  // The tensor-core instance runs long on grids that leave SM slots free
+  // (1024 x 2048 rows x keys at 4 x 8 heads: 256 CTAs of 79 us): serialized
+  // launches would place the next grid's waiting CTAs into those slots at
+  // once, unevenly over the SMs, and that grid then ran 60 % longer.  Plain
+  // launches place a grid on empty SMs (its grid_dep_* calls are no-ops then).
+  if (p.mask_kind == SDPA_MASK_NONE)
     small_d_mma_kernel<false><<<grid, kRowsPerCta, 0, stream>>>(p, hp);
   else
     small_d_mma_kernel<true><<<grid, kRowsPerCta, 0, stream>>>(p, hp);
@@ -929,8 +944,7 @@ cudaError_t launch_split_kv_ws(const Params& p, int* cnt, void* data, cudaStream
   a.ws_ml = static_cast<float2*>(data);
   a.ws_o = reinterpret_cast<float*>(static_cast<char*>(data) + ((nml + 255) & ~size_t(255)));
   dim3 grid((unsigned)a.nsplit, (unsigned)p.Hq, (unsigned)p.B);
-  split_kv_kernel<<<grid, kSplitThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_serialized(split_kv_kernel, grid, dim3(kSplitThreads), 0, stream, a);
 }
 
 template <int NCL>
@@ -952,13 +966,16 @@ static cudaError_t launch_cluster(const Params& p, cudaStream_t stream) {
   cfg.blockDim = dim3(kSplitThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = (unsigned)NCL;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  // programmatic serialization: the kernel waits for the previous grid first
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, split_kv_cluster_kernel<NCL>, a);
 }
 
