@@ -953,19 +953,23 @@ __global__ void __launch_bounds__(kThreads, 1) flash_fwd_tc(const __grid_constan
             }
           }
         }
+        // the other parts' O rows are loaded whether or not the part saw a
+        // key (a part without one may have left its slot unwritten: its rows
+        // are then not added), so the loads need not wait for (m, l)
 #pragma unroll
         for (int k = 0; k < kMaxSplit; ++k) {
-          if (ml[k].y > 0.f) {
-            const float w = ex2_approx(ml[k].x - M);
+          if (k < nsplit && k != sidx) {
+            const bool add = ml[k].y > 0.f;
+            const float w = add ? ex2_approx(ml[k].x - M) : 0.f;
             den = fmaf(w, ml[k].y, den);
             const float4* src = reinterpret_cast<const float4*>(args.ws_o) + (part0 + k) * (D / 4) * 256 + row;
 #pragma unroll
             for (int c = 0; c < D; c += 4) {
               const float4 o4 = __ldcg(src + (c / 4) * 256);
-              acc[c] = fmaf(w, o4.x, acc[c]);
-              acc[c + 1] = fmaf(w, o4.y, acc[c + 1]);
-              acc[c + 2] = fmaf(w, o4.z, acc[c + 2]);
-              acc[c + 3] = fmaf(w, o4.w, acc[c + 3]);
+              acc[c] = add ? fmaf(w, o4.x, acc[c]) : acc[c];
+              acc[c + 1] = add ? fmaf(w, o4.y, acc[c + 1]) : acc[c + 1];
+              acc[c + 2] = add ? fmaf(w, o4.z, acc[c + 2]) : acc[c + 2];
+              acc[c + 3] = add ? fmaf(w, o4.w, acc[c + 3]) : acc[c + 3];
             }
           }
         }
