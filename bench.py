@@ -260,7 +260,13 @@ def n_input_sets(spec: W.Spec) -> int:
     return min(64, max(2, math.ceil(2 * L2_BYTES / max(spec.bytes(), 1))))
 
 
-def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, ws: int, path=0, sets=None):
+def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, ws: int, path=0, sets=None,
+                  per_launch: bool = True):
+    """K launches back to back on the current stream between two CUDA events.
+    ``per_launch`` also brackets every launch with its own pair of events
+    (for a per-launch median).  Those events sit between consecutive
+    launches, so the headline measurement leaves them out: its launches follow
+    one another as a caller's consecutive calls on a stream do."""
     per_set = spec.bytes()
     if sets is None:
         sets = make_device_sets(spec, device, n_input_sets(spec), seed_base=spec.seed + 1000 * rank)
@@ -279,16 +285,18 @@ def time_workload(S, spec: W.Spec, device, steps: int, warmup: int, rank: int, w
     t0 = time.time()
     e0.record(stream)
     for i in range(steps):
-        starts[i].record(stream)
+        if per_launch:
+            starts[i].record(stream)
         launch(S, spec, sets[i % nsets], stream, path)
-        ends[i].record(stream)
+        if per_launch:
+            ends[i].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(device)
     t1 = time.time()
     if ws > 1:
         torch.distributed.barrier()
     total_ms = e0.elapsed_time(e1)
-    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)] if per_launch else [total_ms / steps] * steps
     return dict(total_ms=total_ms, launch_ms=launch_ms, t0=t0, t1=t1, nsets=nsets,
                 set_bytes=per_set)
 
@@ -571,7 +579,9 @@ def run_ours(args):
     sampler = ClockSampler(torch.cuda.current_device() if ws == 1 else local)
     sampler.start()
     time.sleep(0.3)
-    r = time_workload(S, spec, device, args.steps, args.warmup, rank, ws)
+    # one step = one launch; the K steps run back to back between two events,
+    # as a caller's consecutive calls on a stream would
+    r = time_workload(S, spec, device, args.steps, args.warmup, rank, ws, per_launch=False)
     clocks = sampler.summary(r["t0"], r["t1"])
     sampler.stop()
 
