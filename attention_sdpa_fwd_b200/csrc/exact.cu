@@ -103,6 +103,17 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
 
   for (long long j0 = lo; j0 < hi; j0 += 32) {
     const long long j = j0 + lane;
+    const int nk = (int)((hi - j0) < 32 ? (hi - j0) : 32);
+    // one column per lane: the chunk's V column goes out with the K rows, so
+    // the chunk costs one round trip to memory instead of one per KB keys
+    float vcol[CPL == 1 ? 32 : 1];
+    if constexpr (CPL == 1) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const bool live = t < nk && owns_cols && dcheck_kv(p, b, hk, j0 + t);
+        vcol[t] = live ? to_f32(vb[(j0 + t) * p.svt + col0]) : 0.f;
+      }
+    }
     float s = -INFINITY;
     if (j < hi && dcheck_kv(p, b, hk, j)) {
       s = p.scale * (p.k_vec16 ? dot_row<T, D>(qs, kb + j * p.skt) : dot_any<T>(qs, kb + j * p.skt, D));
@@ -126,11 +137,15 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     l = l * corr + psum;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] *= corr;
+    if constexpr (CPL == 1) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) acc[0] = fmaf(__shfl_sync(0xffffffffu, pj, t), vcol[t], acc[0]);
+      m = mnew;
+      continue;
+    }
     // the value sum over the chunk's keys, KB at a time: the KB V loads go
-    // out together, then the FMAs (one round trip per KB keys; 16 when a lane
-    // owns one column)
-    constexpr int KB = CPL == 1 ? 16 : 8;
-    const int nk = (int)((hi - j0) < 32 ? (hi - j0) : 32);
+    // out together, then the FMAs (one round trip per KB keys)
+    constexpr int KB = 8;
     for (int t0 = 0; t0 < nk; t0 += KB) {
       float pt[KB], vv[KB][CPL];
 #pragma unroll
