@@ -45,7 +45,11 @@ __device__ __forceinline__ float dot_any(const float* __restrict__ qs, const T* 
   return acc;
 }
 
-template <typename T, int D>
+// VPRE (one output column per lane only): a chunk's V column is loaded at the
+// top of the chunk, with the K rows (one round trip per chunk), at about twice
+// the registers; the host takes it for launches of at most one wave at that
+// occupancy, where latency, not the number of resident warps, sets the time.
+template <typename T, int D, bool VPRE>
 __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
   // launched behind the previous grid in the stream (programmatic
   // serialization): wait for it before any global-memory access
@@ -106,8 +110,9 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     const int nk = (int)((hi - j0) < 32 ? (hi - j0) : 32);
     // one column per lane: the chunk's V column goes out with the K rows, so
     // the chunk costs one round trip to memory instead of one per KB keys
-    float vcol[CPL == 1 ? 32 : 1];
-    if constexpr (CPL == 1) {
+    constexpr bool kVpre = VPRE && CPL == 1;
+    float vcol[kVpre ? 32 : 1];
+    if constexpr (kVpre) {
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
         const bool live = t < nk && owns_cols && dcheck_kv(p, b, hk, j0 + t);
@@ -137,15 +142,16 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     l = l * corr + psum;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] *= corr;
-    if constexpr (CPL == 1) {
+    if constexpr (kVpre) {
 #pragma unroll
       for (int t = 0; t < 32; ++t) acc[0] = fmaf(__shfl_sync(0xffffffffu, pj, t), vcol[t], acc[0]);
       m = mnew;
       continue;
     }
     // the value sum over the chunk's keys, KB at a time: the KB V loads go
-    // out together, then the FMAs (one round trip per KB keys)
-    constexpr int KB = 8;
+    // out together, then the FMAs (one round trip per KB keys; 16 when a lane
+    // owns one column)
+    constexpr int KB = CPL == 1 ? 16 : 8;
     for (int t0 = 0; t0 < nk; t0 += KB) {
       float pt[KB], vv[KB][CPL];
 #pragma unroll
@@ -175,17 +181,28 @@ __global__ void __launch_bounds__(kWarps * 32) exact_kernel(Params p) {
     p.lse[((long long)b * p.Hq + h) * p.Tq + i] = l > 0.f ? m + logf(l) : -INFINITY;
 }
 
+template <typename T, int D, bool VPRE>
+cudaError_t launch_tv(const Params& p, dim3 grid, size_t smem, cudaStream_t stream) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(exact_kernel<T, D, VPRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_serialized(exact_kernel<T, D, VPRE>, grid, dim3(kWarps * 32), smem, stream, p);
+}
+
 template <typename T, int D>
 cudaError_t launch_t(const Params& p, cudaStream_t stream) {
   const int per_warp = D + (p.use_rel ? (p.kh_n + p.kw_n) : 0);
   const size_t smem = sizeof(float) * (size_t)per_warp * kWarps;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(exact_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
   dim3 grid((unsigned)((p.Tq + kWarps - 1) / kWarps), (unsigned)p.Hq, (unsigned)p.B);
-  return launch_serialized(exact_kernel<T, D>, grid, dim3(kWarps * 32), smem, stream, p);
+  if constexpr (D <= 32) {
+    // the V-column prefetch holds about twice the registers (three CTAs per
+    // SM): taken while the whole grid fits one wave at that occupancy
+    const long long ctas = (long long)grid.x * grid.y * grid.z;
+    if (ctas <= 3LL * num_sms()) return launch_tv<T, D, true>(p, grid, smem, stream);
+  }
+  return launch_tv<T, D, false>(p, grid, smem, stream);
 }
 
 }  // namespace
