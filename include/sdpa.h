@@ -34,6 +34,15 @@
  * Every entry point is asynchronous on `stream` (no host synchronisation)
  * unless stated otherwise, and returns SDPA_OK (0) or a negative sdpa_status.
  * Argument errors are detected on the host before anything is launched.
+ *
+ * Stream order is kept as for any kernel launch.  The attention kernels are
+ * launched with programmatic stream serialization and let the next grid in
+ * the stream be scheduled once all their CTAs have started; each waits for
+ * the grid before it (griddepcontrol.wait) before touching global memory.  A
+ * caller's own kernel that follows on the same stream and is itself launched
+ * with programmatic serialization must likewise wait
+ * (cudaGridDependencySynchronize) before it reads this library's outputs;
+ * kernels launched without that attribute need nothing.
  */
 #ifndef SDPA_H_
 #define SDPA_H_
